@@ -1,0 +1,217 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle of the dense-and-sparse quantized
+ * matrix-vector product
+ *
+ *     y[b][i] = sum_j x[b][j] * What[i][j],   What = W_dense + W_sparse
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark load this file's library.  It shares no code,
+ * header, table or helper with the CUDA library; it is compiled on its own
+ * with gcc and knows nothing of the packed device layout.
+ *
+ * Sources it restates:
+ *  - SqueezeLLM page, "Dense-and-Sparse decomposition": W = W_dense + W_sparse,
+ *    the sparse part being the outliers kept in fp16.
+ *  - SpQR page, "Diagramme de la matrice sparse vs dense": the dense part has
+ *    holes at the outlier positions; the sparse part is CSR with fp16 values.
+ *  - SpQR page, "Le format de stockage sparse": values / col_idx / row_ptr
+ *    (row i owns entries row_ptr[i] .. row_ptr[i+1]-1).
+ *  - SpQR page, "Quantification d'un modele" (wbits 3, groupsize 16): the
+ *    dense part is uniform codes over groups of 16 inputs.  The decode
+ *    formula is not printed; it is read as w = scale * (q - zero), with the
+ *    fp16 scale and the integral fp16 zero of the weight's group.
+ *  - SqueezeLLM page, "Sensitivity-based non-uniform quantization": the dense
+ *    part is codes into a non-uniform table of bins; read as one fp16 table
+ *    of 2^bits centroids per output row, w = table[row][q].
+ *
+ * Precision.  A decoded dense weight is an fp16 value: a table entry is
+ * copied bit for bit; an affine weight is scale*(q-zero) evaluated exactly in
+ * fp64 (an 11-bit significand times a small integer) and rounded once to
+ * fp16, nearest-even.  Everything after decoding is fp64: the outlier is
+ * added to the decoded weight, and y_ref, together with the error scale
+ * bound[b][i] = sum_j |What[i][j]| * |x[b][j]|, is a plain ascending-j sum.
+ *
+ * Pins (tests/test_oracle.py): fp16 conversions against numpy on every
+ * binary16 pattern and on ties; the SpQR CSR worked example; table decode
+ * returning the table; affine decode against hand-computed values; the
+ * product against exact rational arithmetic; degenerate cases.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_LUT 0
+#define ORACLE_AFFINE 1
+#define ORACLE_GROUP 16
+
+/* IEEE 754 binary16 -> real value: sign, 5-bit biased exponent (bias 15),
+ * 10-bit fraction; exponent 0 encodes subnormals m * 2^-24. */
+double oracle_half_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 31;
+    int m = h & 1023;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + m), e - 25);
+    return sign ? -v : v;
+}
+
+/* Real value -> nearest binary16, ties to the even significand; values at or
+ * beyond 65520 become infinity; results below 2^-14 are subnormal. */
+uint16_t oracle_double_to_half(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    int e2, E;
+    double m, fl, r;
+    uint64_t n;
+    if (isnan(v))
+        return 0x7E00;
+    if (isinf(v))
+        return sign | 0x7C00;
+    if (a == 0.0)
+        return sign;
+    frexp(a, &e2);          /* a in [2^(e2-1), 2^e2) */
+    E = e2 - 1;             /* binade of a */
+    if (E < -14)
+        E = -14;            /* subnormal binade shares the quantum 2^-24 */
+    m = ldexp(a, 10 - E);   /* a in units of the quantum 2^(E-10); exact */
+    fl = floor(m);
+    r = m - fl;
+    n = (uint64_t)fl;
+    if (r > 0.5 || (r == 0.5 && (n & 1)))
+        n += 1;
+    if (n == 2048) {        /* rounded up into the next binade */
+        n = 1024;
+        E += 1;
+    }
+    if (E > 15)
+        return sign | 0x7C00;
+    if (n < 1024)           /* only reachable in the subnormal binade */
+        return sign | (uint16_t)n;
+    return sign | (uint16_t)(((E + 15) << 10) | (int)(n - 1024));
+}
+
+void oracle_half_to_double_n(const uint16_t *h, double *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = oracle_half_to_double(h[i]);
+}
+
+void oracle_double_to_half_n(const double *v, uint16_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = oracle_double_to_half(v[i]);
+}
+
+/* Decoded dense weight of row i, column j, as an fp16 bit pattern.
+ * table: LUT mode rows x 2^bits centroids; AFFINE mode rows x cols/16 scales.
+ * zeros: AFFINE mode rows x cols/16 integral zeros (unused in LUT mode). */
+uint16_t oracle_decode_one(int64_t i, int64_t j, int cols, int bits, int mode,
+                           const uint8_t *codes, const uint16_t *table,
+                           const uint16_t *zeros)
+{
+    int q = codes[i * (int64_t)cols + j];
+    if (mode == ORACLE_LUT)
+        return table[i * ((int64_t)1 << bits) + q];
+    {
+        int64_t g = i * (int64_t)(cols / ORACLE_GROUP) + j / ORACLE_GROUP;
+        double scale = oracle_half_to_double(table[g]);
+        double zero = oracle_half_to_double(zeros[g]);
+        return oracle_double_to_half(scale * ((double)q - zero));
+    }
+}
+
+/* W_dense: rows x cols fp16 bit patterns (holes decode from their codes). */
+void oracle_decode(int rows, int cols, int bits, int mode, const uint8_t *codes,
+                   const uint16_t *table, const uint16_t *zeros, uint16_t *wd)
+{
+    for (int64_t i = 0; i < rows; i++)
+        for (int64_t j = 0; j < cols; j++)
+            wd[i * cols + j] =
+                oracle_decode_one(i, j, cols, bits, mode, codes, table, zeros);
+}
+
+/* What row i in fp64: decoded dense weights, then each CSR entry of the row
+ * added to the weight at its column. */
+void oracle_weight_row(int64_t i, int cols, int bits, int mode,
+                       const uint8_t *codes, const uint16_t *table,
+                       const uint16_t *zeros, const int32_t *row_ptr,
+                       const int32_t *col_idx, const uint16_t *values,
+                       double *wrow)
+{
+    for (int64_t j = 0; j < cols; j++)
+        wrow[j] = oracle_half_to_double(
+            oracle_decode_one(i, j, cols, bits, mode, codes, table, zeros));
+    for (int64_t k = row_ptr[i]; k < row_ptr[i + 1]; k++)
+        wrow[col_idx[k]] += oracle_half_to_double(values[k]);
+}
+
+/* What: rows x cols fp64. */
+void oracle_materialize(int rows, int cols, int bits, int mode,
+                        const uint8_t *codes, const uint16_t *table,
+                        const uint16_t *zeros, const int32_t *row_ptr,
+                        const int32_t *col_idx, const uint16_t *values,
+                        double *w)
+{
+    for (int64_t i = 0; i < rows; i++)
+        oracle_weight_row(i, cols, bits, mode, codes, table, zeros, row_ptr,
+                          col_idx, values, w + i * cols);
+}
+
+/* y_ref and bound for the listed output rows only (all rows when
+ * row_list == NULL, n_list == rows).  x: batch x cols fp16; y_ref and bound:
+ * batch x n_list fp64, column t holding row row_list[t]. */
+int oracle_gemv_rows(int rows, int cols, int bits, int mode,
+                     const uint8_t *codes, const uint16_t *table,
+                     const uint16_t *zeros, const int32_t *row_ptr,
+                     const int32_t *col_idx, const uint16_t *values, int batch,
+                     const uint16_t *x, const int32_t *row_list, int n_list,
+                     double *y_ref, double *bound)
+{
+    double *wrow = (double *)malloc(sizeof(double) * (cols > 0 ? cols : 1));
+    double *xd = (double *)malloc(sizeof(double) * ((int64_t)batch * cols + 1));
+    if (!wrow || !xd) {
+        free(wrow);
+        free(xd);
+        return -1;
+    }
+    for (int64_t t = 0; t < (int64_t)batch * cols; t++)
+        xd[t] = oracle_half_to_double(x[t]);
+    for (int t = 0; t < n_list; t++) {
+        int64_t i = row_list ? row_list[t] : t;
+        oracle_weight_row(i, cols, bits, mode, codes, table, zeros, row_ptr,
+                          col_idx, values, wrow);
+        for (int b = 0; b < batch; b++) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t j = 0; j < cols; j++) {
+                acc += wrow[j] * xd[(int64_t)b * cols + j];
+                mag += fabs(wrow[j]) * fabs(xd[(int64_t)b * cols + j]);
+            }
+            y_ref[(int64_t)b * n_list + t] = acc;
+            bound[(int64_t)b * n_list + t] = mag;
+        }
+    }
+    (void)rows;
+    free(wrow);
+    free(xd);
+    return 0;
+}
+
+/* Full product: y_ref, bound are batch x rows. */
+int oracle_gemv(int rows, int cols, int bits, int mode, const uint8_t *codes,
+                const uint16_t *table, const uint16_t *zeros,
+                const int32_t *row_ptr, const int32_t *col_idx,
+                const uint16_t *values, int batch, const uint16_t *x,
+                double *y_ref, double *bound)
+{
+    return oracle_gemv_rows(rows, cols, bits, mode, codes, table, zeros,
+                            row_ptr, col_idx, values, batch, x, NULL, rows,
+                            y_ref, bound);
+}

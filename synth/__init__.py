@@ -1,0 +1,333 @@
+"""Seeded synthetic workloads for the dense-and-sparse quantized GEMV.
+
+This module only *produces inputs*: the logical dense codes with their
+per-row lookup tables or per-group scale/zero pairs, the CSR outliers and the
+fp16 activations.  It never decodes a weight and never forms a product, so it
+holds none of the arithmetic that the oracle and the CUDA path compute; both
+of them consume what it returns.
+
+What the workloads imitate (all draws come from ``numpy.random.default_rng``):
+
+* Base weights ``W ~ N(0, 0.02^2)`` in fp64, then Laplace(0, 0.2) spikes added
+  at the chosen outlier positions (SpQR page, "Qu'est-ce qu'un poids outlier ?":
+  a Gaussian bulk with a few very large weights).
+* The outliers leave the dense part (they become holes, "trous") and go to a
+  CSR store of fp16 values with column indices and row pointers (SpQR page,
+  "Le format de stockage sparse"; SqueezeLLM page, "Dense-and-Sparse
+  decomposition", W = W_dense + W_sparse).  The stored value is the original
+  weight rounded to fp16.
+* Dense part, one of two encodings:
+  - ``lut``: SqueezeLLM-style non-uniform bins, one fp16 table of 2^bits
+    centroids per output row (SqueezeLLM page, "Sensitivity-based
+    non-uniform quantization").  The centroids are the row's odd quantiles
+    (2k+1)/2^(bits+1) of its non-hole weights; each weight takes the nearest
+    centroid (ties to the lower index), a hole takes the centroid nearest 0.
+  - ``affine``: SpQR-style uniform codes over groups of 16 input columns
+    (SpQR page, quant_config "wbits" and "groupsize": 16) with an fp16 scale
+    and an integral fp16 zero per group; ``w ~ scale * (q - zero)``.  The range
+    of a group is widened to contain 0 so that holes encode exactly.
+* ``x ~ N(0, 1)`` rounded to fp16, drawn after everything else.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+LUT = "lut"
+AFFINE = "affine"
+GROUP = 16
+
+
+def round_half_up(v: float) -> int:
+    return int(math.floor(v + 0.5))
+
+
+def f16_bits(a) -> np.ndarray:
+    """fp64 values -> fp16 bit patterns (numpy's round-to-nearest-even)."""
+    return np.asarray(a, dtype=np.float64).astype(np.float16).view(np.uint16)
+
+
+@dataclasses.dataclass
+class Problem:
+    """One quantized layer plus activations, in logical (unpacked) form.
+
+    codes   uint8  [rows, cols]          one code per weight, < 2^bits
+    table   uint16 [rows, 2^bits]        lut: fp16 centroids of each row
+            uint16 [rows, cols/16]       affine: fp16 scale of each group
+    zeros   uint16 [rows, cols/16]       affine: fp16 integral zero; lut: None
+    row_ptr int32  [rows+1]              CSR row pointers
+    col_idx int32  [nnz]                 CSR column indices, increasing per row
+    values  uint16 [nnz]                 CSR fp16 outlier values
+    x       uint16 [batch, cols]         fp16 activations
+    """
+    name: str
+    rows: int
+    cols: int
+    bits: int
+    mode: str
+    codes: np.ndarray
+    table: np.ndarray
+    zeros: Optional[np.ndarray]
+    row_ptr: np.ndarray
+    col_idx: np.ndarray
+    values: np.ndarray
+    x: np.ndarray
+
+    @property
+    def nnz(self) -> int:
+        return int(self.row_ptr[-1])
+
+    @property
+    def batch(self) -> int:
+        return int(self.x.shape[0])
+
+    def with_x(self, x: np.ndarray) -> "Problem":
+        return dataclasses.replace(self, x=np.ascontiguousarray(x, dtype=np.uint16))
+
+    def canonical_bytes(self, batch: Optional[int] = None) -> int:
+        """Bytes one product moves under the canonical accounting: packed
+        codes, fp16 table or fp16 scale + fp16 zero, CSR as fp16 value +
+        int32 column + int32 row pointer, fp16 x and y."""
+        b = self.batch if batch is None else batch
+        codes = self.rows * self.cols * self.bits // 8
+        if self.mode == LUT:
+            meta = self.rows * (1 << self.bits) * 2
+        else:
+            meta = self.rows * (self.cols // GROUP) * 4
+        csr = self.nnz * 6 + (self.rows + 1) * 4
+        return codes + meta + csr + b * self.cols * 2 + b * self.rows * 2
+
+
+# ---------------------------------------------------------------- outliers
+
+def _distinct_cells(rng, n_want: int, draw, taken: set) -> List[int]:
+    """Draw flat cell indices with ``draw(k)`` until n_want new distinct ones
+    (not already in ``taken``) are collected; collisions are redrawn."""
+    out: List[int] = []
+    while len(out) < n_want:
+        cand = draw(max(2 * (n_want - len(out)), 16))
+        for c in cand.tolist():
+            if c not in taken:
+                taken.add(c)
+                out.append(c)
+                if len(out) == n_want:
+                    break
+    return out
+
+
+def _structured_positions(rng, M: int, N: int, nnz: int) -> np.ndarray:
+    """Half of the outliers in 2% of rows and 2% of columns, half uniform."""
+    rows_sel = rng.choice(M, math.ceil(0.02 * M), replace=False)
+    cols_sel = rng.choice(N, math.ceil(0.02 * N), replace=False)
+    n_struct = nnz // 2
+    n_rowpart = n_struct // 2
+    n_colpart = n_struct - n_rowpart
+    n_uniform = nnz - n_struct
+    taken: set = set()
+    pos = _distinct_cells(
+        rng, n_rowpart,
+        lambda k: rows_sel[rng.integers(0, len(rows_sel), k)] * N + rng.integers(0, N, k),
+        taken)
+    pos += _distinct_cells(
+        rng, n_colpart,
+        lambda k: rng.integers(0, M, k) * N + cols_sel[rng.integers(0, len(cols_sel), k)],
+        taken)
+    pos += _distinct_cells(rng, n_uniform, lambda k: rng.integers(0, M * N, k), taken)
+    return np.asarray(pos, dtype=np.int64)
+
+
+def zipf_row_counts(rng, M: int, N: int, nnz: int, alpha: float = 1.2) -> np.ndarray:
+    """Per-row outlier counts proportional to rank^-alpha for a seeded random
+    ranking of the rows, summing to nnz, each clipped at N (the excess of a
+    clipped row is spread over the unclipped rows; leftover units go to the
+    largest fractional remainders)."""
+    rank = np.empty(M, dtype=np.int64)
+    rank[rng.permutation(M)] = np.arange(1, M + 1)
+    w = rank.astype(np.float64) ** (-alpha)
+    if nnz > M * N:
+        raise ValueError("more outliers than cells")
+    target = np.zeros(M, dtype=np.float64)
+    clipped = np.zeros(M, dtype=bool)
+    remaining = float(nnz)
+    for _ in range(M + 1):
+        free = ~clipped
+        share = w[free] / w[free].sum() * remaining
+        over = share > N
+        if not over.any():
+            target[free] = share
+            break
+        idx = np.flatnonzero(free)[over]
+        target[idx] = N
+        clipped[idx] = True
+        remaining = nnz - target[clipped].sum()
+    counts = np.floor(target).astype(np.int64)
+    left = nnz - int(counts.sum())
+    if left > 0:
+        rem = target - counts
+        rem[counts >= N] = -1.0
+        order = np.argsort(-rem, kind="stable")
+        counts[order[:left]] += 1
+    assert counts.sum() == nnz and counts.max() <= N
+    return counts
+
+
+def _zipf_positions(rng, M: int, N: int, nnz: int) -> np.ndarray:
+    counts = zipf_row_counts(rng, M, N, nnz)
+    pos = []
+    for r in range(M):
+        if counts[r]:
+            pos.append(r * N + np.sort(rng.choice(N, int(counts[r]), replace=False)))
+    return np.concatenate(pos).astype(np.int64) if pos else np.zeros(0, np.int64)
+
+
+# ---------------------------------------------------------------- dense part
+
+def _quantize_lut(Wd: np.ndarray, hole: np.ndarray, bits: int):
+    M, N = Wd.shape
+    K = 1 << bits
+    levels = (2.0 * np.arange(K) + 1.0) / (2.0 * K)
+    table = np.zeros((M, K), dtype=np.uint16)
+    codes = np.zeros((M, N), dtype=np.uint8)
+    chunk = max(1, (1 << 22) // max(1, N * K))
+    for r0 in range(0, M, chunk):
+        r1 = min(M, r0 + chunk)
+        cent = np.zeros((r1 - r0, K), dtype=np.float64)
+        for r in range(r0, r1):
+            vals = Wd[r][~hole[r]]
+            if vals.size:
+                cent[r - r0] = np.quantile(vals, levels)
+        tb = f16_bits(cent)
+        table[r0:r1] = tb
+        c16 = tb.view(np.float16).astype(np.float64)
+        w = np.where(hole[r0:r1], 0.0, Wd[r0:r1])
+        dist = np.abs(w[:, :, None] - c16[:, None, :])
+        codes[r0:r1] = np.argmin(dist, axis=2).astype(np.uint8)
+    return codes, table
+
+
+def _quantize_affine(Wd: np.ndarray, bits: int):
+    M, N = Wd.shape
+    qmax = (1 << bits) - 1
+    G = Wd.reshape(M, N // GROUP, GROUP)
+    mn = np.minimum(G.min(axis=2), 0.0)
+    mx = np.maximum(G.max(axis=2), 0.0)
+    s16 = f16_bits((mx - mn) / qmax)
+    sval = s16.view(np.float16).astype(np.float64)
+    degenerate = ~(np.isfinite(sval) & (sval > 0))
+    sval = np.where(degenerate, 1.0, sval)
+    s16 = np.where(degenerate, np.uint16(0x3C00), s16).astype(np.uint16)
+    zero = np.clip(np.rint(-mn / sval), 0, qmax)
+    zero = np.where(degenerate, 0.0, zero)
+    q = np.rint(G / sval[:, :, None]) + zero[:, :, None]
+    codes = np.clip(q, 0, qmax).astype(np.uint8).reshape(M, N)
+    return codes, s16, f16_bits(zero)
+
+
+# ---------------------------------------------------------------- assembly
+
+def make_problem(rows: int, cols: int, bits: int, mode: str, density: float,
+                 outliers: str = "uniform", seed: int = 0, batch: int = 1,
+                 name: str = "") -> Problem:
+    """Build one layer: outlier kind is 'topk', 'uniform', 'structured',
+    'zipf' or 'none'."""
+    if cols % GROUP:
+        raise ValueError("cols must be a multiple of 16")
+    M, N = rows, cols
+    rng = np.random.default_rng(seed)
+    W = rng.normal(0.0, 0.02, size=(M, N))
+    nnz = round_half_up(density * M * N) if outliers != "none" else 0
+    Wf = W.reshape(-1)
+    if nnz == 0:
+        pos = np.zeros(0, dtype=np.int64)
+    elif outliers in ("topk", "uniform"):
+        spike_pos = rng.choice(M * N, nnz, replace=False)
+        Wf[spike_pos] += rng.laplace(0.0, 0.2, nnz)
+        if outliers == "topk":
+            pos = np.argsort(-np.abs(Wf), kind="stable")[:nnz]
+        else:
+            pos = spike_pos
+    elif outliers == "structured":
+        pos = _structured_positions(rng, M, N, nnz)
+        Wf[pos] += rng.laplace(0.0, 0.2, nnz)
+    elif outliers == "zipf":
+        pos = _zipf_positions(rng, M, N, nnz)
+        Wf[pos] += rng.laplace(0.0, 0.2, nnz)
+    else:
+        raise ValueError(outliers)
+    pos = np.sort(np.asarray(pos, dtype=np.int64))
+    values = f16_bits(Wf[pos])
+    r_of = pos // N
+    col_idx = (pos % N).astype(np.int32)
+    row_ptr = np.zeros(M + 1, dtype=np.int32)
+    np.add.at(row_ptr, r_of + 1, 1)
+    row_ptr = np.cumsum(row_ptr).astype(np.int32)
+    hole = np.zeros((M, N), dtype=bool)
+    hole.reshape(-1)[pos] = True
+    Wd = np.where(hole, 0.0, W)
+    del W, Wf
+    if mode == LUT:
+        codes, table = _quantize_lut(Wd, hole, bits)
+        zeros = None
+    elif mode == AFFINE:
+        codes, table, zeros = _quantize_affine(Wd, bits)
+    else:
+        raise ValueError(mode)
+    x = f16_bits(rng.normal(0.0, 1.0, size=(batch, N)))
+    return Problem(name=name, rows=M, cols=N, bits=bits, mode=mode, codes=codes,
+                   table=table, zeros=zeros, row_ptr=row_ptr, col_idx=col_idx,
+                   values=values, x=x)
+
+
+# ---------------------------------------------------------------- the five workloads
+
+C4_LAYERS = (("q", 6656, 6656), ("k", 6656, 6656), ("v", 6656, 6656),
+             ("o", 6656, 6656), ("gate", 17920, 6656), ("up", 17920, 6656),
+             ("down", 6656, 17920))
+
+CONFIGS: Dict[str, dict] = {
+    "c0": dict(rows=1024, cols=1024, bits=3, mode=LUT, density=0.01,
+               outliers="topk", seed=0, batches=(1,),
+               about="1024x1024 3-bit row-LUT, 1% top-|w| outliers after Laplace spikes"),
+    "c1": dict(rows=4096, cols=4096, bits=3, mode=LUT, density=0.0045,
+               outliers="uniform", seed=1, batches=(1,),
+               about="4096x4096 3-bit row-LUT, 0.45% uniform outliers"),
+    "c2": dict(rows=11008, cols=4096, bits=3, mode=AFFINE, density=0.01,
+               outliers="structured", seed=2, batches=(1,),
+               about="11008x4096 3-bit affine g16, 1% structured outliers"),
+    "c3": dict(rows=4096, cols=11008, bits=4, mode=LUT, density=0.005,
+               outliers="zipf", seed=3, batches=(1, 2, 4, 8),
+               about="4096x11008 4-bit row-LUT, 0.5% Zipf(1.2) row-skewed outliers"),
+}
+
+
+def config_names() -> List[str]:
+    return ["c0", "c1", "c2", "c3"] + ["c4_" + n for n, _, _ in C4_LAYERS]
+
+
+def make_config(name: str, batch: Optional[int] = None) -> Problem:
+    """Workload by name: c0..c3, or c4_<layer> for the seven linear layers of
+    the 6656-hidden / 17920-FFN block.  The activations hold the largest batch
+    of the config's sweep (8 for c3, 16 for c4) unless ``batch`` is given;
+    smaller batches take the leading rows."""
+    if name.startswith("c4_"):
+        layer = name[3:]
+        for li, (ln, M, N) in enumerate(C4_LAYERS):
+            if ln == layer:
+                return make_problem(M, N, 3, AFFINE, 0.01, "uniform", 40 + li,
+                                    16 if batch is None else batch, name)
+        raise KeyError(name)
+    c = CONFIGS[name]
+    b = max(c["batches"]) if batch is None else batch
+    return make_problem(c["rows"], c["cols"], c["bits"], c["mode"], c["density"],
+                        c["outliers"], c["seed"], b, name)
+
+
+def describe(name: str) -> str:
+    if name.startswith("c4_"):
+        for ln, M, N in C4_LAYERS:
+            if "c4_" + ln == name:
+                return f"{M}x{N} 3-bit affine g16, 1% uniform outliers ({ln} of the 33B-scale block)"
+    return CONFIGS[name]["about"]
