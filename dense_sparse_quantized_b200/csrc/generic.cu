@@ -1,0 +1,165 @@
+// generic.cu -- the reference-quality CUDA path: one warp per output row,
+// every weight decoded to its fp16 value exactly as dsq_decode writes it,
+// fp32 accumulation, CSR outliers added by the same warp, y written once.
+// Serves every shape, mode and batch; the tuned kernels replace it on the
+// shapes they cover.  Also dsq_decode's kernel.
+#include "internal.h"
+
+namespace dsq {
+
+// Code of column c (0..31) of a slot from its code words w[0..BITS-1].
+template <int BITS>
+__device__ __forceinline__ uint32_t slot_code(const uint32_t (&w)[4], int c) {
+    uint32_t q = 0;
+#pragma unroll
+    for (int k = 0; k < BITS; k++) {
+        int wi, pos;
+        code_bit_place(BITS, c, k, &wi, &pos);
+        q |= ((w[wi] >> pos) & 1u) << k;
+    }
+    return q;
+}
+
+template <int BITS, int MODE>
+__device__ __forceinline__ void load_slot(const MatrixView &m, const uint32_t *rec, int s,
+                                          uint32_t (&w)[4], uint32_t &scales, uint32_t &zb) {
+#pragma unroll
+    for (int p = 0; p < BITS; p++) w[p] = __ldg(rec + code_word_index(BITS, MODE, m.slots, s, p));
+    if (MODE == DSQ_MODE_AFFINE_G16) {
+        scales = __ldg(rec + scale_word_index(BITS, m.slots, s));
+        zb = __ldg((const uint8_t *)(rec + zero_word_offset(BITS, MODE, m.slots)) + s);
+    }
+}
+
+// fp16 value of the decoded dense weight (bits as an unsigned short).
+template <int MODE>
+__device__ __forceinline__ __half decode_weight(const __half *row_table, uint32_t q,
+                                                uint32_t scales, uint32_t zb, int c) {
+    if (MODE == DSQ_MODE_LUT_ROW) return row_table[q];
+    int e = c >> 4;  // group inside the slot
+    __half s = __ushort_as_half((unsigned short)(scales >> (16 * e)));
+    int z = (int)((zb >> (4 * e)) & 15u);
+    // (q - z) is a small integer and s has an 11-bit significand: the fp32
+    // product is exact, so this is the single rounding of s*(q-z) to fp16.
+    return __float2half_rn(__half2float(s) * (float)((int)q - z));
+}
+
+template <int BITS, int MODE, int BC>
+__global__ void __launch_bounds__(256) gemv_generic_kernel(MatrixView m, const __half *__restrict__ x,
+                                                           __half *__restrict__ y, int batch, int b0) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= m.rows) return;
+    const int nb = min(BC, batch - b0);
+    const int N = m.cols;
+    const uint32_t *rec = m.dense + (size_t)row * m.row_words;
+    const __half *row_table = MODE == DSQ_MODE_LUT_ROW ? (const __half *)m.table + ((size_t)row << BITS) : nullptr;
+    float acc[BC];
+#pragma unroll
+    for (int b = 0; b < BC; b++) acc[b] = 0.f;
+
+    for (int s = lane; s < m.slots; s += 32) {
+        uint32_t w[4] = {0, 0, 0, 0}, scales = 0, zb = 0;
+        load_slot<BITS, MODE>(m, rec, s, w, scales, zb);
+#pragma unroll
+        for (int c = 0; c < 32; c++) {
+            const int j = s * 32 + c;
+            if (j < N) {
+                float wv = __half2float(decode_weight<MODE>(row_table, slot_code<BITS>(w, c), scales, zb, c));
+#pragma unroll
+                for (int b = 0; b < BC; b++)
+                    if (b < nb) acc[b] = fmaf(wv, __half2float(x[(size_t)(b0 + b) * N + j]), acc[b]);
+            }
+        }
+    }
+    const int k0 = m.row_ptr[row], k1 = m.row_ptr[row + 1];
+    for (int k = k0 + lane; k < k1; k += 32) {
+        const float v = __half2float(__ushort_as_half(m.val[k]));
+        const int j = m.col[k];
+#pragma unroll
+        for (int b = 0; b < BC; b++)
+            if (b < nb) acc[b] = fmaf(v, __half2float(x[(size_t)(b0 + b) * N + j]), acc[b]);
+    }
+#pragma unroll
+    for (int b = 0; b < BC; b++) {
+        float a = acc[b];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0 && b < nb) y[(size_t)(b0 + b) * m.rows + row] = __float2half_rn(a);
+    }
+}
+
+template <int BITS, int MODE>
+__global__ void decode_kernel(MatrixView m, __half *__restrict__ w_out) {
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= (int64_t)m.rows * m.slots) return;
+    const int row = (int)(t / m.slots), s = (int)(t % m.slots);
+    const uint32_t *rec = m.dense + (size_t)row * m.row_words;
+    const __half *row_table = MODE == DSQ_MODE_LUT_ROW ? (const __half *)m.table + ((size_t)row << BITS) : nullptr;
+    uint32_t w[4] = {0, 0, 0, 0}, scales = 0, zb = 0;
+    load_slot<BITS, MODE>(m, rec, s, w, scales, zb);
+#pragma unroll
+    for (int c = 0; c < 32; c++) {
+        const int j = s * 32 + c;
+        if (j < m.cols)
+            w_out[(size_t)row * m.cols + j] = decode_weight<MODE>(row_table, slot_code<BITS>(w, c), scales, zb, c);
+    }
+}
+
+__global__ void zero_kernel(__half *y, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        y[i] = __ushort_as_half(0);
+}
+
+template <int BITS, int MODE>
+static void launch_generic_t(const MatrixView &m, const __half *x, __half *y, int batch, cudaStream_t st) {
+    const int warps = 8;
+    dim3 grid((m.rows + warps - 1) / warps);
+    for (int b0 = 0; b0 < batch; b0 += 8) {
+        int nb = batch - b0;
+        if (nb == 1)
+            gemv_generic_kernel<BITS, MODE, 1><<<grid, warps * 32, 0, st>>>(m, x, y, batch, b0);
+        else if (nb <= 4)
+            gemv_generic_kernel<BITS, MODE, 4><<<grid, warps * 32, 0, st>>>(m, x, y, batch, b0);
+        else
+            gemv_generic_kernel<BITS, MODE, 8><<<grid, warps * 32, 0, st>>>(m, x, y, batch, b0);
+    }
+}
+
+int launch_gemv_generic(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t st) {
+    const MatrixView &m = h->view;
+    if (m.rows == 0) return DSQ_OK;
+    if (m.cols == 0) return launch_zero(y, (int64_t)batch * m.rows, st);
+    if (m.bits == 3 && m.mode == 0) launch_generic_t<3, 0>(m, x, y, batch, st);
+    else if (m.bits == 4 && m.mode == 0) launch_generic_t<4, 0>(m, x, y, batch, st);
+    else if (m.bits == 3) launch_generic_t<3, 1>(m, x, y, batch, st);
+    else launch_generic_t<4, 1>(m, x, y, batch, st);
+    return cudaGetLastError() == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+}
+
+int gemv_launch_count(const dsq_handle_s *h, int batch) {
+    if (h->view.rows == 0) return 0;
+    if (h->view.cols == 0) return 1;
+    return (batch + 7) / 8;
+}
+
+int launch_decode(const dsq_handle_s *h, __half *w, cudaStream_t st) {
+    const MatrixView &m = h->view;
+    const int64_t n = (int64_t)m.rows * m.slots;
+    if (n == 0) return DSQ_OK;
+    const int threads = 256;
+    const unsigned grid = (unsigned)((n + threads - 1) / threads);
+    if (m.bits == 3 && m.mode == 0) decode_kernel<3, 0><<<grid, threads, 0, st>>>(m, w);
+    else if (m.bits == 4 && m.mode == 0) decode_kernel<4, 0><<<grid, threads, 0, st>>>(m, w);
+    else if (m.bits == 3) decode_kernel<3, 1><<<grid, threads, 0, st>>>(m, w);
+    else decode_kernel<4, 1><<<grid, threads, 0, st>>>(m, w);
+    return cudaGetLastError() == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+}
+
+int launch_zero(__half *y, int64_t n, cudaStream_t st) {
+    if (n <= 0) return DSQ_OK;
+    zero_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(y, n);
+    return cudaGetLastError() == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+}
+
+}  // namespace dsq

@@ -1,0 +1,116 @@
+// layout.h -- the packed blob written by dsq_pack and read by the kernels.
+//
+// The blob is a 256-byte header followed by 256-byte-aligned sections:
+//
+//   dense    rows x row_words u32: one "row record" per output row
+//   table    LUT_ROW only: rows x 2^bits fp16 centroids, as given
+//   row_ptr  int32 [rows+1]
+//   col      uint16 [nnz]   CSR column indices (cols <= 65535)
+//   val      fp16   [nnz]   CSR outlier values
+//
+// Row record.  The columns of a row are cut into S = ceil(cols/32) "slots"
+// of 32 consecutive columns; the tail slot is padded with code 0 (and, in
+// affine mode, scale 0 / zero 0 for the padded group).  One slot carries
+// 32 codes in `bits` u32 code words.  Within a record, per mode:
+//
+//   LUT_ROW, 3 bit:    3 planes of S words: word p of slot s at [p*S + s]
+//   LUT_ROW, 4 bit:    S uint4 (4 code words) at [4s .. 4s+3]
+//   AFFINE_G16, 3 bit: S uint4 = (code word 0, 1, 2, scale pair) at [4s..]
+//   AFFINE_G16, 4 bit: S uint4 code words, then S scale-pair words at [4S+s]
+//   AFFINE_G16:        then S zero bytes (byte s = zero[2s] | zero[2s+1]<<4)
+//                      starting at word Z = (bits == 3 ? 4S : 5S)
+//
+// and the record is padded to a multiple of 4 words, so every record and
+// every uint4 starts on a 16-byte boundary.  A scale pair is
+// scale[2s] | scale[2s+1] << 16 (the two groups of 16 in the slot).
+//
+// Code bits inside a slot.  4-bit: column c in word c/8, bits 4(c%8)..+3.
+// 3-bit: columns are placed so that every field the kernels mask lies in
+// bits 0..22 of a word, or of the word shifted right by 9 -- an fp32 whose
+// exponent field is zero is then the code times 2^-149 exactly (see the
+// kernels).  Column c < 30: word c/10, t = c%10, field at 3t (t < 7) or at
+// 21 + 3(t-7) (t >= 7).  Column 30: bits 0,1 at word 0 bits 30,31 and bit 2
+// at word 1 bit 30.  Column 31: bit 0 at word 1 bit 31, bits 1,2 at word 2
+// bits 30,31.
+#pragma once
+#include <stdint.h>
+
+#ifndef __CUDACC__
+#define __host__
+#define __device__
+#endif
+
+namespace dsq {
+
+constexpr char kMagic[8] = {'D', 'S', 'Q', 'B', 'L', 'O', 'B', '1'};
+constexpr uint32_t kVersion = 1;
+constexpr uint32_t kHeaderBytes = 256;
+constexpr uint64_t kSectionAlign = 256;
+constexpr int kSlotCols = 32;
+constexpr int kGroup = 16;
+
+struct BlobHeader {
+    char magic[8];
+    uint32_t version;
+    uint32_t header_bytes;
+    int32_t rows, cols, bits, mode;
+    int64_t nnz;
+    int32_t slots;      // S
+    int32_t row_words;  // u32 words per row record (multiple of 4)
+    uint64_t off_dense, off_table, off_row_ptr, off_col, off_val, total;
+    uint8_t reserved[kHeaderBytes - 8 - 4 - 4 - 16 - 8 - 8 - 48];
+};
+static_assert(sizeof(BlobHeader) == kHeaderBytes, "header size");
+
+__host__ __device__ inline int slots_of(int cols) { return (cols + kSlotCols - 1) / kSlotCols; }
+
+// Word offset (inside a record) of the zero bytes; -1 in LUT mode.
+__host__ __device__ inline int zero_word_offset(int bits, int mode, int S) {
+    return mode == 1 ? (bits == 3 ? 4 * S : 5 * S) : -1;
+}
+
+__host__ __device__ inline int row_words_of(int bits, int mode, int S) {
+    int w;
+    if (mode == 0)
+        w = bits * S;
+    else
+        w = zero_word_offset(bits, mode, S) + (S + 3) / 4;
+    return (w + 3) & ~3;
+}
+
+// Position of bit k (0 = least significant) of column c's code inside a
+// slot: returns the code word index (0..bits-1) and the bit position.
+__host__ __device__ inline void code_bit_place(int bits, int c, int k, int *word, int *pos) {
+    if (bits == 4) {
+        *word = c >> 3;
+        *pos = 4 * (c & 7) + k;
+        return;
+    }
+    if (c < 30) {
+        int t = c % 10;
+        *word = c / 10;
+        *pos = (t < 7 ? 3 * t : 21 + 3 * (t - 7)) + k;
+        return;
+    }
+    if (c == 30) {
+        if (k < 2) { *word = 0; *pos = 30 + k; }
+        else       { *word = 1; *pos = 30; }
+        return;
+    }
+    // c == 31
+    if (k == 0) { *word = 1; *pos = 31; }
+    else        { *word = 2; *pos = 29 + k; }
+}
+
+// Word index (inside a record) of code word p of slot s.
+__host__ __device__ inline int code_word_index(int bits, int mode, int S, int s, int p) {
+    if (bits == 3 && mode == 0) return p * S + s;
+    return 4 * s + p;
+}
+
+// Word index of the scale pair of slot s (affine only).
+__host__ __device__ inline int scale_word_index(int bits, int S, int s) {
+    return bits == 3 ? 4 * s + 3 : 4 * S + s;
+}
+
+}  // namespace dsq

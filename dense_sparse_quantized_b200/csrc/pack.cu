@@ -1,0 +1,195 @@
+// pack.cu -- dsq_pack / dsq_blob_desc: host-side validation of the logical
+// weights and their layout into the packed blob (see layout.h).
+#include <math.h>
+#include <string.h>
+
+#include <vector>
+
+#include "../../include/dsq.h"
+#include "layout.h"
+#include "internal.h"
+
+namespace dsq {
+
+// IEEE binary16 bit pattern -> double (host; validation only).
+double half_bits_to_double(uint16_t h) {
+    int e = (h >> 10) & 31, m = h & 1023;
+    double v = e == 0 ? ldexp((double)m, -24)
+             : e == 31 ? (m ? NAN : INFINITY)
+                       : ldexp((double)(1024 + m), e - 25);
+    return (h & 0x8000) ? -v : v;
+}
+
+static inline uint64_t align_up(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
+
+int check_desc(const dsq_desc *d) {
+    if (!d) return DSQ_ERR_INVALID_ARG;
+    if (d->rows < 0 || d->cols < 0 || d->cols % kGroup != 0) return DSQ_ERR_INVALID_ARG;
+    if (d->bits != 3 && d->bits != 4) return DSQ_ERR_INVALID_ARG;
+    if (d->mode != DSQ_MODE_LUT_ROW && d->mode != DSQ_MODE_AFFINE_G16) return DSQ_ERR_INVALID_ARG;
+    if (d->nnz < 0 || d->nnz > (int64_t)d->rows * d->cols) return DSQ_ERR_INVALID_ARG;
+    if (d->cols > 65535) return DSQ_ERR_UNSUPPORTED;
+    return DSQ_OK;
+}
+
+void plan_blob(const dsq_desc *d, BlobHeader *h) {
+    memset(h, 0, sizeof(*h));
+    memcpy(h->magic, kMagic, sizeof(kMagic));
+    h->version = kVersion;
+    h->header_bytes = kHeaderBytes;
+    h->rows = d->rows;
+    h->cols = d->cols;
+    h->bits = d->bits;
+    h->mode = d->mode;
+    h->nnz = d->nnz;
+    h->slots = slots_of(d->cols);
+    h->row_words = row_words_of(d->bits, d->mode, h->slots);
+    uint64_t off = kHeaderBytes;
+    h->off_dense = off;
+    off = align_up(off + (uint64_t)d->rows * h->row_words * 4, kSectionAlign);
+    h->off_table = off;
+    if (d->mode == DSQ_MODE_LUT_ROW)
+        off = align_up(off + (uint64_t)d->rows * (1u << d->bits) * 2, kSectionAlign);
+    h->off_row_ptr = off;
+    off = align_up(off + (uint64_t)(d->rows + 1) * 4, kSectionAlign);
+    h->off_col = off;
+    off = align_up(off + (uint64_t)d->nnz * 2, kSectionAlign);
+    h->off_val = off;
+    off = align_up(off + (uint64_t)d->nnz * 2, kSectionAlign);
+    h->total = off;
+}
+
+int parse_blob(const void *packed, size_t bytes, BlobHeader *out) {
+    if (!packed || bytes < kHeaderBytes) return DSQ_ERR_INVALID_ARG;
+    BlobHeader h;
+    memcpy(&h, packed, sizeof(h));
+    if (memcmp(h.magic, kMagic, sizeof(kMagic)) != 0 || h.version != kVersion ||
+        h.header_bytes != kHeaderBytes)
+        return DSQ_ERR_INVALID_ARG;
+    dsq_desc d = {h.rows, h.cols, h.bits, h.mode, h.nnz};
+    int rc = check_desc(&d);
+    if (rc != DSQ_OK) return rc;
+    BlobHeader want;
+    plan_blob(&d, &want);
+    if (want.slots != h.slots || want.row_words != h.row_words || want.off_dense != h.off_dense ||
+        want.off_table != h.off_table || want.off_row_ptr != h.off_row_ptr ||
+        want.off_col != h.off_col || want.off_val != h.off_val || want.total != h.total ||
+        h.total > bytes)
+        return DSQ_ERR_INVALID_ARG;
+    *out = h;
+    return DSQ_OK;
+}
+
+}  // namespace dsq
+
+using namespace dsq;
+
+extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t *table,
+                        const uint16_t *zeros, const int32_t *row_ptr, const int32_t *col_idx,
+                        const uint16_t *values, void *out, size_t *out_bytes) {
+    if (!out_bytes) return DSQ_ERR_INVALID_ARG;
+    int rc = check_desc(d);
+    if (rc != DSQ_OK) return rc;
+    const int64_t M = d->rows, N = d->cols, nnz = d->nnz;
+    const int bits = d->bits, mode = d->mode, K = 1 << bits, qmax = K - 1;
+    const int64_t G = N / kGroup;
+    const bool any = M * N > 0;
+    if (any && !codes) return DSQ_ERR_INVALID_ARG;
+    if (M > 0 && (mode == DSQ_MODE_LUT_ROW || G > 0) && !table) return DSQ_ERR_INVALID_ARG;
+    if (mode == DSQ_MODE_LUT_ROW && zeros) return DSQ_ERR_INVALID_ARG;
+    if (mode == DSQ_MODE_AFFINE_G16 && any && !zeros) return DSQ_ERR_INVALID_ARG;
+    if (M > 0 && !row_ptr) return DSQ_ERR_INVALID_ARG;
+    if (nnz > 0 && (!col_idx || !values)) return DSQ_ERR_INVALID_ARG;
+
+    // ---- validate every input before writing anything
+    for (int64_t t = 0; t < M * N; t++)
+        if (codes[t] > qmax) return DSQ_ERR_INVALID_ARG;
+    if (mode == DSQ_MODE_LUT_ROW) {
+        for (int64_t t = 0; t < M * K; t++)
+            if (!isfinite(half_bits_to_double(table[t]))) return DSQ_ERR_INVALID_ARG;
+    } else {
+        for (int64_t t = 0; t < M * G; t++) {
+            double s = half_bits_to_double(table[t]);
+            double z = half_bits_to_double(zeros[t]);
+            if (!isfinite(s) || !(z >= 0 && z <= qmax) || z != floor(z)) return DSQ_ERR_INVALID_ARG;
+            double span = fabs(s) * (z > qmax - z ? z : qmax - z);
+            if (!(span < 65520.0)) return DSQ_ERR_INVALID_ARG;
+        }
+    }
+    if (M > 0) {
+        if (row_ptr[0] != 0 || row_ptr[M] != nnz) return DSQ_ERR_INVALID_ARG;
+        for (int64_t i = 0; i < M; i++) {
+            if (row_ptr[i + 1] < row_ptr[i]) return DSQ_ERR_INVALID_ARG;
+            for (int64_t k = row_ptr[i]; k < row_ptr[i + 1]; k++) {
+                if (col_idx[k] < 0 || col_idx[k] >= N) return DSQ_ERR_INVALID_ARG;
+                if (k > row_ptr[i] && col_idx[k] <= col_idx[k - 1]) return DSQ_ERR_INVALID_ARG;
+            }
+        }
+    } else if (nnz != 0) {
+        return DSQ_ERR_INVALID_ARG;
+    }
+    for (int64_t k = 0; k < nnz; k++)
+        if (!isfinite(half_bits_to_double(values[k]))) return DSQ_ERR_INVALID_ARG;
+
+    BlobHeader h;
+    plan_blob(d, &h);
+    if (!out || *out_bytes < h.total) {
+        *out_bytes = h.total;
+        return DSQ_ERR_BUFFER_TOO_SMALL;
+    }
+    *out_bytes = h.total;
+    uint8_t *blob = (uint8_t *)out;
+    memset(blob, 0, h.total);
+    memcpy(blob, &h, sizeof(h));
+
+    // ---- dense row records
+    const int S = h.slots;
+    int place_word[32][4], place_pos[32][4];
+    for (int c = 0; c < 32; c++)
+        for (int k = 0; k < bits; k++) code_bit_place(bits, c, k, &place_word[c][k], &place_pos[c][k]);
+    for (int64_t i = 0; i < M; i++) {
+        uint32_t *rec = (uint32_t *)(blob + h.off_dense) + i * h.row_words;
+        for (int s = 0; s < S; s++) {
+            uint32_t w[4] = {0, 0, 0, 0};
+            for (int c = 0; c < 32; c++) {
+                int64_t j = (int64_t)s * 32 + c;
+                if (j >= N) break;
+                uint32_t q = codes[i * N + j];
+                for (int k = 0; k < bits; k++)
+                    w[place_word[c][k]] |= ((q >> k) & 1u) << place_pos[c][k];
+            }
+            for (int p = 0; p < bits; p++) rec[code_word_index(bits, mode, S, s, p)] = w[p];
+            if (mode == DSQ_MODE_AFFINE_G16) {
+                uint32_t pair = 0, zb = 0;
+                for (int e = 0; e < 2; e++) {
+                    int64_t g = 2 * (int64_t)s + e;
+                    if (g >= G) break;
+                    pair |= (uint32_t)table[i * G + g] << (16 * e);
+                    zb |= (uint32_t)half_bits_to_double(zeros[i * G + g]) << (4 * e);
+                }
+                rec[scale_word_index(bits, S, s)] = pair;
+                ((uint8_t *)(rec + zero_word_offset(bits, mode, S)))[s] = (uint8_t)zb;
+            }
+        }
+    }
+    if (mode == DSQ_MODE_LUT_ROW && M > 0) memcpy(blob + h.off_table, table, (size_t)M * K * 2);
+    if (M > 0) memcpy(blob + h.off_row_ptr, row_ptr, (size_t)(M + 1) * 4);
+    else memset(blob + h.off_row_ptr, 0, 4);
+    uint16_t *col = (uint16_t *)(blob + h.off_col);
+    for (int64_t k = 0; k < nnz; k++) col[k] = (uint16_t)col_idx[k];
+    if (nnz > 0) memcpy(blob + h.off_val, values, (size_t)nnz * 2);
+    return DSQ_OK;
+}
+
+extern "C" int dsq_blob_desc(const void *packed, size_t bytes, dsq_desc *out) {
+    if (!out) return DSQ_ERR_INVALID_ARG;
+    BlobHeader h;
+    int rc = parse_blob(packed, bytes, &h);
+    if (rc != DSQ_OK) return rc;
+    out->rows = h.rows;
+    out->cols = h.cols;
+    out->bits = h.bits;
+    out->mode = h.mode;
+    out->nnz = h.nnz;
+    return DSQ_OK;
+}

@@ -1,0 +1,180 @@
+/*
+ * dsq.h -- C ABI of libdsq: the dense-and-sparse quantized matrix-vector /
+ * skinny-matrix product on one NVIDIA B200 (sm_100a).
+ *
+ *     y[b][i] = sum_j x[b][j] * What[i][j],   What = W_dense + W_sparse
+ *
+ * W_dense (SqueezeLLM page, "Dense-and-Sparse decomposition"; SpQR page,
+ * "Diagramme de la matrice sparse vs dense") holds one 3- or 4-bit code per
+ * weight, decoded either
+ *   - DSQ_MODE_LUT_ROW:    w = table[i][q], a per-output-row table of 2^bits
+ *                          fp16 centroids (SqueezeLLM page, "Sensitivity-based
+ *                          non-uniform quantization"), or
+ *   - DSQ_MODE_AFFINE_G16: w = fp16(scale[i][g] * (q - zero[i][g])), g = j/16,
+ *                          an fp16 scale and an integral fp16 zero per group
+ *                          of 16 inputs (SpQR page, quant_config "wbits",
+ *                          "groupsize": 16; the formula is this library's
+ *                          reading, the page prints none).
+ * At the positions of the outliers the dense part holds "holes" whose codes
+ * still decode (to 0 when the encoder chose q = zero).
+ * W_sparse holds the outliers as fp16 CSR: values / col_idx / row_ptr (SpQR
+ * page, "Le format de stockage sparse"); each outlier is ADDED to the decoded
+ * dense weight at its position.
+ *
+ * Conventions for every call:
+ *  - Return value is a dsq_status (0 = DSQ_OK); nothing else reports errors.
+ *    No call aborts, traps or throws.  dsq_status_string() names a code.
+ *  - "host" pointers are ordinary CPU memory; "device" pointers are CUDA
+ *    global memory on the handle's device.  fp16 data is passed as raw IEEE
+ *    binary16 bit patterns (uint16_t or void*).
+ *  - A cudaStream_t is passed as void* (NULL = the legacy default stream),
+ *    so this header needs no CUDA header.
+ *  - Work on a stream is asynchronous: a DSQ_OK from dsq_gemv/dsq_decode
+ *    means the kernels were launched; a fault inside them shows up at the
+ *    caller's next synchronisation, as with any CUDA call.
+ */
+#ifndef DSQ_H
+#define DSQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSQ_API __attribute__((visibility("default")))
+#else
+#define DSQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSQ_OK = 0,
+    DSQ_ERR_INVALID_ARG = -1,     /* a NULL pointer, a size or value out of range, a malformed blob */
+    DSQ_ERR_UNSUPPORTED = -2,     /* well-formed but outside this build (e.g. cols > 65535) */
+    DSQ_ERR_CUDA = -3,            /* a CUDA runtime call or a kernel launch failed */
+    DSQ_ERR_OOM = -4,             /* device allocation failed */
+    DSQ_ERR_BUFFER_TOO_SMALL = -5,/* output buffer smaller than required; size reported */
+    DSQ_ERR_DEVICE = -6           /* a kernel reported an error through its status word */
+} dsq_status;
+
+enum { DSQ_MODE_LUT_ROW = 0, DSQ_MODE_AFFINE_G16 = 1 };
+
+/* Shape and encoding of one quantized weight matrix (rows = out features M,
+ * cols = in features N).  Requirements: rows >= 0; cols >= 0 and
+ * cols % 16 == 0; cols <= 65535 (column indices are stored in 16 bits);
+ * bits in {3, 4}; mode one of DSQ_MODE_*; 0 <= nnz <= rows*cols. */
+typedef struct {
+    int32_t rows;
+    int32_t cols;
+    int32_t bits;
+    int32_t mode;
+    int64_t nnz;
+} dsq_desc;
+
+typedef struct dsq_handle_s *dsq_handle_t;
+
+/*
+ * dsq_pack -- validate the logical (unpacked) weights and write the packed
+ * blob that dsq_create uploads.  Host-only; thread-safe; touches no GPU.
+ *
+ *   d        host; shape and encoding.
+ *   codes    host uint8 [rows][cols] row-major, one code per byte, < 2^bits.
+ *   table    host fp16.  LUT_ROW: [rows][2^bits] centroids.  AFFINE_G16:
+ *            [rows][cols/16] scales.  All finite.
+ *   zeros    host fp16 [rows][cols/16] (AFFINE_G16: integral values in
+ *            [0, 2^bits-1]); must be NULL for LUT_ROW.  For AFFINE_G16,
+ *            |scale| * max(zero, 2^bits-1-zero) must stay below 65520 so
+ *            every decoded weight is finite.
+ *   row_ptr  host int32 [rows+1]: row_ptr[0] = 0, nondecreasing,
+ *            row_ptr[rows] = nnz.
+ *   col_idx  host int32 [nnz]: < cols, strictly increasing inside a row.
+ *   values   host fp16 [nnz], finite.
+ *   out      host buffer of *out_bytes bytes, or NULL to query the size.
+ *   out_bytes in: capacity of out; out: bytes required (always written when
+ *            the inputs are valid).
+ * Returns DSQ_OK, DSQ_ERR_INVALID_ARG (first invalid input; nothing written
+ * to out), DSQ_ERR_UNSUPPORTED, or DSQ_ERR_BUFFER_TOO_SMALL (out too small
+ * or NULL; *out_bytes holds the size).  The blob is position-independent
+ * plain bytes and may be stored and reloaded.  With rows*cols == 0 the
+ * pointers of empty arrays may be NULL.
+ */
+DSQ_API int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t *table,
+             const uint16_t *zeros, const int32_t *row_ptr,
+             const int32_t *col_idx, const uint16_t *values, void *out,
+             size_t *out_bytes);
+
+/*
+ * dsq_blob_desc -- read the shape of a packed blob (host).  Returns
+ * DSQ_ERR_INVALID_ARG when the blob is not one dsq_pack wrote.
+ */
+DSQ_API int dsq_blob_desc(const void *packed, size_t bytes, dsq_desc *out);
+
+/*
+ * dsq_create -- upload a packed blob to CUDA device `device` and build the
+ * row-tile schedule for that device's SM count.  The handle owns every
+ * device allocation it makes (released by dsq_destroy); the blob stays the
+ * caller's and may be freed on return.  Synchronous.  The calling thread's
+ * current device is left unchanged.
+ * Returns DSQ_OK, DSQ_ERR_INVALID_ARG (NULL out, malformed blob, bad
+ * device), DSQ_ERR_UNSUPPORTED (not an sm_100 device), DSQ_ERR_OOM or
+ * DSQ_ERR_CUDA.
+ */
+DSQ_API int dsq_create(const void *packed, size_t bytes, int device, dsq_handle_t *out);
+
+/*
+ * dsq_gemv -- y[b][i] = sum_j x[b][j] * What[i][j] for b < batch.
+ *   x      device fp16 [batch][cols], row-major, 16-byte aligned (may be
+ *          NULL only when cols == 0).
+ *   y      device fp16 [batch][rows], row-major, 16-byte aligned (may be
+ *          NULL only when rows == 0); fully overwritten, each
+ *          element written once, rounded to nearest from an fp32 sum.
+ *   batch  >= 1.  Batches of 16 and more go through the tensor-core path.
+ *   stream cudaStream_t of the handle's device, as void*.
+ * x and y are the caller's and must not overlap.  The handle is read-only
+ * here, so calls on several streams or threads may run concurrently.
+ * Accuracy: |y - y_exact| <= 1e-3 * sum_j |What[i][j]| * |x[b][j]|.
+ * Returns DSQ_OK, DSQ_ERR_INVALID_ARG (NULL or misaligned pointer,
+ * batch < 1) or DSQ_ERR_CUDA (launch failure).
+ */
+DSQ_API int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void *stream);
+
+/*
+ * dsq_gemv_launches -- number of kernel launches one dsq_gemv call of this
+ * batch makes on this handle (0 for an empty matrix); -1 for a NULL handle
+ * or batch < 1.  Host-only.
+ */
+DSQ_API int dsq_gemv_launches(dsq_handle_t h, int batch);
+
+/*
+ * dsq_decode -- write W_dense (no outliers added) as fp16
+ * [rows][cols] row-major to device memory w_dense_out (caller-owned), bit
+ * for bit equal to the definitions above.  A test hook; asynchronous on
+ * `stream`.
+ */
+DSQ_API int dsq_decode(dsq_handle_t h, void *w_dense_out, void *stream);
+
+/*
+ * dsq_handle_desc -- shape of the matrix a handle holds (host).
+ */
+DSQ_API int dsq_handle_desc(dsq_handle_t h, dsq_desc *out);
+
+/*
+ * dsq_device_bytes -- device bytes the handle holds (packed weights, CSR,
+ * schedule), for accounting.  Returns 0 for NULL.
+ */
+DSQ_API size_t dsq_device_bytes(dsq_handle_t h);
+
+/* dsq_destroy -- free the handle's device memory; NULL is a no-op.  The
+ * caller must make sure no work using the handle is still in flight. */
+DSQ_API int dsq_destroy(dsq_handle_t h);
+
+/* Static, never-NULL text for a status code. */
+DSQ_API const char *dsq_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSQ_H */

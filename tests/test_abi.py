@@ -1,0 +1,252 @@
+"""Host-side checks of the C ABI: the library loads, exports what include/*.h
+declares, validates inputs with the documented status codes, and lays out the
+blob as layout.h describes.  No GPU and no kernel launch."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import dense_sparse_quantized_b200 as dsq
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        for m in re.finditer(r"^DSQ_API\s+[\w\s\*]+?\b(dsq_\w+)\s*\(", open(h).read(), re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert {"dsq_pack", "dsq_create", "dsq_gemv", "dsq_decode", "dsq_destroy",
+            "dsq_status_string"} <= names
+    out = subprocess.run(["nm", "-D", "--defined-only", dsq.LIBRARY], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (dsq_\w+)", out))
+    assert names <= exported, names - exported
+    lib = dsq.library()
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_status_strings():
+    for s in (0, -1, -2, -3, -4, -5, -6, 99):
+        assert isinstance(dsq.status_string(s), str) and dsq.status_string(s)
+
+
+def test_null_handle_calls_are_rejected_on_the_host():
+    lib = dsq.library()
+    assert lib.dsq_gemv(None, None, None, 1, None) == dsq.DSQ_ERR_INVALID_ARG
+    assert lib.dsq_decode(None, None, None) == dsq.DSQ_ERR_INVALID_ARG
+    assert lib.dsq_destroy(None) == dsq.DSQ_OK
+    assert lib.dsq_device_bytes(None) == 0
+    assert lib.dsq_create(None, 0, 0, None) == dsq.DSQ_ERR_INVALID_ARG
+
+
+# --------------------------------------------------------------- validation
+
+def small(bits=3, mode="affine", rows=5, cols=48, seed=0, density=0.05):
+    return synth.make_problem(rows, cols, bits, mode, density, "uniform", seed, 1)
+
+
+def pack_status(p, **over):
+    a = dict(rows=p.rows, cols=p.cols, bits=p.bits, mode=p.mode, codes=p.codes,
+             table=p.table, zeros=p.zeros, row_ptr=p.row_ptr, col_idx=p.col_idx,
+             values=p.values)
+    a.update(over)
+    try:
+        dsq.pack(**a)
+        return dsq.DSQ_OK
+    except dsq.DSQError as e:
+        return e.status
+
+
+def test_pack_accepts_valid_inputs():
+    for bits in (3, 4):
+        for mode in ("lut", "affine"):
+            assert pack_status(small(bits, mode)) == dsq.DSQ_OK
+
+
+@pytest.mark.parametrize("case", [
+    "bits2", "bits5", "cols_not16", "bad_mode", "code_too_big", "zeros_for_lut",
+    "no_zeros_affine", "zero_not_integral", "zero_too_big", "scale_nan", "scale_overflow",
+    "table_inf", "rowptr_start", "rowptr_end", "rowptr_decreasing", "col_unsorted",
+    "col_duplicate", "col_out_of_range", "col_negative", "value_nan", "null_codes"])
+def test_pack_rejects(case):
+    p = small(3, "affine")
+    pl = small(3, "lut")
+    bad = dict(
+        bits2=(p, dict(bits=2)), bits5=(p, dict(bits=5)),
+        cols_not16=(p, dict(cols=40)), bad_mode=(p, dict(mode=7)),
+        code_too_big=(p, dict(codes=np.where(np.arange(p.codes.size).reshape(p.codes.shape) == 7, 8, p.codes))),
+        zeros_for_lut=(pl, dict(zeros=np.zeros((5, 3), np.uint16))),
+        no_zeros_affine=(p, dict(zeros=None)),
+        zero_not_integral=(p, dict(zeros=np.full_like(p.zeros, 0x3800))),   # 0.5
+        zero_too_big=(p, dict(zeros=np.full_like(p.zeros, 0x4800))),        # 8
+        scale_nan=(p, dict(table=np.full_like(p.table, 0x7E00))),
+        scale_overflow=(p, dict(table=np.full_like(p.table, 0x7400))),      # 16384 * max(z, 7-z) >= 65536
+        table_inf=(pl, dict(table=np.full_like(pl.table, 0x7C00))),
+        rowptr_start=(p, dict(row_ptr=p.row_ptr + 1)),
+        rowptr_end=(p, dict(row_ptr=np.concatenate([p.row_ptr[:-1], [p.row_ptr[-1] + 1]]))),
+        rowptr_decreasing=(p, dict(row_ptr=np.array([0, 3, 2, 5, 5, p.row_ptr[-1]]))),
+        col_unsorted=(p, dict(col_idx=p.col_idx[::-1].copy())),
+        col_duplicate=(p, dict(col_idx=np.where(np.arange(p.nnz) == 1, p.col_idx[0], p.col_idx))),
+        col_out_of_range=(p, dict(col_idx=np.where(np.arange(p.nnz) == p.nnz - 1, 48, p.col_idx))),
+        col_negative=(p, dict(col_idx=np.where(np.arange(p.nnz) == 0, -1, p.col_idx))),
+        value_nan=(p, dict(values=np.full_like(p.values, 0x7E00))),
+        null_codes=(p, dict(codes=None)),
+    )[case]
+    assert pack_status(bad[0], **bad[1]) == dsq.DSQ_ERR_INVALID_ARG
+
+
+def test_pack_unsupported_width():
+    lib = dsq.library()
+    d = dsq.Desc(1, 65536, 3, 1, 0)
+    size = ctypes.c_size_t(0)
+    assert lib.dsq_pack(ctypes.byref(d), None, None, None, None, None, None, None,
+                        ctypes.byref(size)) == dsq.DSQ_ERR_UNSUPPORTED
+
+
+def test_pack_size_query_and_small_buffer():
+    p = small()
+    lib = dsq.library()
+    d = dsq.Desc(p.rows, p.cols, p.bits, 1, p.nnz)
+    arrs = [np.ascontiguousarray(a) for a in (p.codes, p.table, p.zeros)] + \
+           [np.ascontiguousarray(p.row_ptr, np.int32), np.ascontiguousarray(p.col_idx, np.int32),
+            np.ascontiguousarray(p.values)]
+    size = ctypes.c_size_t(0)
+    rc = lib.dsq_pack(ctypes.byref(d), *[a.ctypes.data for a in arrs], None, ctypes.byref(size))
+    assert rc == dsq.DSQ_ERR_BUFFER_TOO_SMALL and size.value > 0
+    need = size.value
+    buf = ctypes.create_string_buffer(need)
+    size = ctypes.c_size_t(need - 1)
+    rc = lib.dsq_pack(ctypes.byref(d), *[a.ctypes.data for a in arrs], buf, ctypes.byref(size))
+    assert rc == dsq.DSQ_ERR_BUFFER_TOO_SMALL and size.value == need
+
+
+def test_blob_desc_and_corruption():
+    p = small(4, "lut")
+    blob = dsq.pack_problem(p)
+    d = dsq.blob_desc(blob)
+    assert (d.rows, d.cols, d.bits, d.mode, d.nnz) == (5, 48, 4, 0, p.nnz)
+    bad = bytearray(blob)
+    bad[0] ^= 0xFF
+    with pytest.raises(dsq.DSQError):
+        dsq.blob_desc(bytes(bad))
+    with pytest.raises(dsq.DSQError):
+        dsq.blob_desc(blob[:100])
+
+
+def test_empty_shapes_pack():
+    for rows, cols in ((0, 16), (3, 0), (0, 0)):
+        blob = dsq.pack(rows, cols, 3, "affine", np.zeros((rows, cols), np.uint8),
+                        np.zeros((rows, cols // 16), np.uint16), np.zeros((rows, cols // 16), np.uint16),
+                        np.zeros(rows + 1, np.int32), np.zeros(0, np.int32), np.zeros(0, np.uint16))
+        d = dsq.blob_desc(blob)
+        assert (d.rows, d.cols, d.nnz) == (rows, cols, 0)
+
+
+# --------------------------------------------------------------- layout round trip
+
+def unpack_blob(blob: bytes):
+    """Test-only reader of the blob, written from the layout description:
+    returns codes, table/scales, zeros, row_ptr, col_idx, values."""
+    b = np.frombuffer(blob, dtype=np.uint8)
+    hdr = np.frombuffer(blob[:96], dtype=np.uint8)
+    rows, cols, bits, mode = np.frombuffer(blob[16:32], np.int32)
+    nnz = int(np.frombuffer(blob[32:40], np.int64)[0])
+    S, row_words = np.frombuffer(blob[40:48], np.int32)
+    off_dense, off_table, off_rp, off_col, off_val, total = np.frombuffer(blob[48:96], np.uint64)
+    rec = np.frombuffer(blob[int(off_dense):int(off_dense) + rows * row_words * 4],
+                        np.uint32).reshape(rows, row_words)
+
+    def place(c, k):
+        if bits == 4:
+            return c // 8, 4 * (c % 8) + k
+        if c < 30:
+            t = c % 10
+            return c // 10, (3 * t if t < 7 else 21 + 3 * (t - 7)) + k
+        if c == 30:
+            return (0, 30 + k) if k < 2 else (1, 30)
+        return (1, 31) if k == 0 else (2, 29 + k)
+
+    codes = np.zeros((rows, cols), np.uint8)
+    for s in range(S):
+        for p_ in range(bits):
+            pass
+        words = [rec[:, (p_ * S + s) if (bits == 3 and mode == 0) else (4 * s + p_)]
+                 for p_ in range(bits)]
+        for c in range(32):
+            j = 32 * s + c
+            if j >= cols:
+                break
+            q = np.zeros(rows, np.uint32)
+            for k in range(bits):
+                wi, pos = place(c, k)
+                q |= ((words[wi] >> np.uint32(pos)) & np.uint32(1)) << np.uint32(k)
+            codes[:, j] = q
+    G = cols // 16
+    if mode == 0:
+        table = np.frombuffer(blob[int(off_table):int(off_table) + rows * (1 << bits) * 2],
+                              np.uint16).reshape(rows, 1 << bits)
+        zeros = None
+    else:
+        table = np.zeros((rows, G), np.uint16)
+        zeros = np.zeros((rows, G), np.uint16)
+        zoff = (4 * S if bits == 3 else 5 * S) * 4
+        for s in range(S):
+            pair = rec[:, 4 * s + 3] if bits == 3 else rec[:, 4 * S + s]
+            zb = rec.view(np.uint8)[:, zoff + s]
+            for e in range(2):
+                g = 2 * s + e
+                if g < G:
+                    table[:, g] = (pair >> np.uint32(16 * e)) & np.uint32(0xFFFF)
+                    zeros[:, g] = np.asarray((zb >> (4 * e)) & 15, np.float64).astype(np.float16).view(np.uint16)
+    row_ptr = np.frombuffer(blob[int(off_rp):int(off_rp) + (rows + 1) * 4], np.int32)
+    col = np.frombuffer(blob[int(off_col):int(off_col) + nnz * 2], np.uint16).astype(np.int32)
+    val = np.frombuffer(blob[int(off_val):int(off_val) + nnz * 2], np.uint16)
+    assert total == len(blob)
+    return codes, table, zeros, row_ptr, col, val
+
+
+@pytest.mark.parametrize("bits,mode,cols", [(3, "lut", 48), (4, "lut", 80), (3, "affine", 48),
+                                            (4, "affine", 112), (3, "affine", 1024), (3, "lut", 16)])
+def test_layout_round_trip(bits, mode, cols):
+    p = synth.make_problem(7, cols, bits, mode, 0.03, "uniform", 2, 1)
+    codes, table, zeros, rp, ci, va = unpack_blob(dsq.pack_problem(p))
+    assert np.array_equal(codes, p.codes)
+    assert np.array_equal(table, p.table)
+    if mode == "affine":
+        assert np.array_equal(zeros, p.zeros)
+    assert np.array_equal(rp, p.row_ptr) and np.array_equal(ci, p.col_idx)
+    assert np.array_equal(va, p.values)
+
+
+def test_three_bit_fields_sit_below_bit_23():
+    """Every 3-bit field is either inside bits 0..22 of its word or inside bits
+    0..22 after a right shift by 9 (the kernels turn a masked field into an
+    exact fp32 subnormal)."""
+    import itertools
+    seen = set()
+    for c in range(32):
+        for k in range(3):
+            if c < 30:
+                t = c % 10
+                pos = (3 * t if t < 7 else 21 + 3 * (t - 7)) + k
+                word = c // 10
+            elif c == 30:
+                word, pos = (0, 30 + k) if k < 2 else (1, 30)
+            else:
+                word, pos = (1, 31) if k == 0 else (2, 29 + k)
+            assert pos <= 22 or 0 <= pos - 9 <= 22
+            assert (word, pos) not in seen
+            seen.add((word, pos))
+    assert len(seen) == 96

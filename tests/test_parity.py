@@ -1,0 +1,242 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Decode: the device's decoded W_dense is bit-identical to the oracle's.
+Product: |y - y_ref| <= 1e-3 * bound element by element, bound =
+sum_j |What[i][j]| * |x[b][j]|; where bound is 0, y is exactly 0.  The
+tolerance covers the fp16 rounding of y (<= 2^-11 |y|), the use of exact
+rather than fp16-rounded affine weights inside the group sums (<= 2^-11 per
+weight, i.e. <= 4.9e-4 * bound) and fp32 accumulation.
+"""
+import numpy as np
+import pytest
+
+import dense_sparse_quantized_b200 as dsq
+import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def to_dev(bits: np.ndarray):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.float16).cuda()
+
+
+def to_bits(t) -> np.ndarray:
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def check_y(y_bits, y_ref, bound, what=""):
+    y = y_bits.view(np.float16).astype(np.float64)
+    assert np.all(np.isfinite(y)), what
+    zero = bound == 0
+    assert np.all(y[zero] == 0), what
+    if (~zero).any():
+        ratio = np.abs(y[~zero] - y_ref[~zero]) / bound[~zero]
+        assert ratio.max() <= TOL, (what, float(ratio.max()))
+        return float(ratio.max())
+    return 0.0
+
+
+def gemv(h, x_bits, batch):
+    x = to_dev(x_bits[:batch])
+    y = h.gemv(x)
+    torch.cuda.synchronize()
+    return to_bits(y)
+
+
+_cache = {}
+
+
+def config(name):
+    if name not in _cache:
+        p = synth.make_config(name)
+        _cache[name] = (p, dsq.Handle(dsq.pack_problem(p)))
+    return _cache[name]
+
+
+def sample_rows(p, n=768, seed=0):
+    """A sample of rows that always holds the first, the last and the rows
+    with the most outliers, plus random ones."""
+    rng = np.random.default_rng(seed)
+    counts = np.diff(p.row_ptr)
+    heavy = np.argsort(-counts, kind="stable")[:64]
+    rnd = rng.choice(p.rows, min(n, p.rows), replace=False)
+    return np.unique(np.concatenate([[0, p.rows - 1], heavy, rnd])).astype(np.int32)
+
+
+# ------------------------------------------------------------- full-size configs
+
+SMALL_CONFIGS = ["c0", "c1", "c2", "c3"]
+C4 = ["c4_" + n for n, _, _ in synth.C4_LAYERS]
+
+
+@pytest.mark.parametrize("name", SMALL_CONFIGS + C4)
+def test_decode_bit_exact(orc, name):
+    p, h = config(name)
+    got = to_bits(h.decode())
+    want = orc.decode(p)
+    mism = np.count_nonzero(got != want)
+    assert mism == 0, f"{mism} decoded weights differ"
+
+
+@pytest.mark.parametrize("name,batch", [("c0", 1), ("c1", 1), ("c2", 1), ("c3", 1), ("c3", 2),
+                                        ("c3", 4), ("c3", 8)])
+def test_gemv_full_oracle(orc, name, batch):
+    p, h = config(name)
+    y = gemv(h, p.x, batch)
+    y_ref, bound = orc.gemv(p, x=p.x[:batch])
+    check_y(y, y_ref, bound, f"{name} B={batch}")
+
+
+@pytest.mark.parametrize("name", C4)
+@pytest.mark.parametrize("batch", [1, 16])
+def test_gemv_c4_sampled(orc, name, batch):
+    p, h = config(name)
+    y = gemv(h, p.x, batch)
+    rows = sample_rows(p, 512)
+    y_ref, bound = orc.gemv(p, x=p.x[:batch], rows=rows)
+    check_y(y[:, rows], y_ref, bound, f"{name} B={batch}")
+
+
+# ------------------------------------------------------------- small shapes
+
+SHAPES = [(1, 16), (7, 48), (64, 1024), (7, 16), (1, 1024), (64, 48), (33, 4096), (130, 80)]
+
+
+@pytest.mark.parametrize("bits,mode", [(3, "lut"), (4, "lut"), (3, "affine"), (4, "affine")])
+@pytest.mark.parametrize("rows,cols", SHAPES)
+def test_small_shapes(orc, bits, mode, rows, cols):
+    p = synth.make_problem(rows, cols, bits, mode, 0.02, "uniform", rows * 7 + cols, 3)
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        assert np.array_equal(to_bits(h.decode()), orc.decode(p))
+        for batch in (1, 2, 3):
+            y = gemv(h, p.x, batch)
+            y_ref, bound = orc.gemv(p, x=p.x[:batch])
+            check_y(y, y_ref, bound, f"{rows}x{cols} {bits} {mode} B={batch}")
+
+
+@pytest.mark.parametrize("mode", ["lut", "affine"])
+@pytest.mark.parametrize("batch", [1, 2, 3, 4, 5, 8, 15, 16, 17, 31, 32, 40])
+def test_batches(orc, mode, batch):
+    p = synth.make_problem(96, 272, 3, mode, 0.02, "uniform", 123, batch)
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        y = gemv(h, p.x, batch)
+        y_ref, bound = orc.gemv(p)
+        check_y(y, y_ref, bound, f"{mode} B={batch}")
+
+
+# ------------------------------------------------------------- edge cases
+
+def edited(p, **kw):
+    import dataclasses
+    return dataclasses.replace(p, **kw)
+
+
+@pytest.mark.parametrize("mode", ["lut", "affine"])
+def test_empty_csr(orc, mode):
+    p = synth.make_problem(50, 256, 3, mode, 0.0, "none", 4, 2)
+    assert p.nnz == 0
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        y_ref, bound = orc.gemv(p)
+        check_y(gemv(h, p.x, 2), y_ref, bound, "empty csr")
+
+
+@pytest.mark.parametrize("mode", ["lut", "affine"])
+def test_all_outlier_rows(orc, mode):
+    """Row 3 has an outlier on every column (nnz = N); row 10 likewise; the
+    other rows keep their outliers."""
+    p = synth.make_problem(20, 96, 4, mode, 0.01, "uniform", 5, 2)
+    rng = np.random.default_rng(1)
+    rows = []
+    for i in range(p.rows):
+        if i in (3, 10):
+            rows.append(np.arange(96))
+        else:
+            rows.append(p.col_idx[p.row_ptr[i]:p.row_ptr[i + 1]])
+    counts = np.array([len(r) for r in rows])
+    rp = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    ci = np.concatenate(rows).astype(np.int32)
+    va = synth.f16_bits(rng.laplace(0, 0.2, ci.size))
+    q = edited(p, row_ptr=rp, col_idx=ci, values=va)
+    with dsq.Handle(dsq.pack_problem(q)) as h:
+        y_ref, bound = orc.gemv(q)
+        check_y(gemv(h, q.x, 2), y_ref, bound, "all-outlier rows")
+
+
+@pytest.mark.parametrize("name", ["c2", "c3"])
+def test_zero_and_one_hot_x(orc, name):
+    p, h = config(name)
+    x0 = np.zeros((1, p.cols), np.uint16)
+    y = gemv(h, x0, 1).view(np.float16)
+    assert np.all(y == 0)
+    hit = np.zeros(p.cols, bool)
+    hit[p.col_idx] = True
+    j = int(np.flatnonzero(~hit)[0]) if (~hit).any() else 0
+    e = np.zeros((1, p.cols), np.uint16)
+    e[0, j] = 0x3C00
+    y = gemv(h, e, 1)
+    y_ref, bound = orc.gemv(p, x=e)
+    check_y(y, y_ref, bound, "one-hot")
+    if not hit[j]:
+        # y_i = W_dense[i][j] exactly: one product, no rounding beyond fp16.
+        wd = orc.decode(p)[:, j]
+        assert np.array_equal(y[0].view(np.float16).astype(np.float64),
+                              wd.view(np.float16).astype(np.float64))
+
+
+def test_degenerate_shapes():
+    for rows, cols in ((0, 32), (5, 0)):
+        blob = dsq.pack(rows, cols, 3, "affine", np.zeros((rows, cols), np.uint8),
+                        np.zeros((rows, cols // 16), np.uint16),
+                        np.zeros((rows, cols // 16), np.uint16), np.zeros(rows + 1, np.int32),
+                        np.zeros(0, np.int32), np.zeros(0, np.uint16))
+        with dsq.Handle(blob) as h:
+            x = torch.randn(2, max(cols, 1), device="cuda").half()[:, :cols].contiguous()
+            y = torch.full((2, rows), 7.0, device="cuda").half()
+            h.gemv(x if cols else torch.empty((2, 0), device="cuda", dtype=torch.float16), y)
+            torch.cuda.synchronize()
+            assert torch.all(y == 0)
+
+
+def test_y_written_in_place_only(orc):
+    """y is written exactly in its [batch, rows] box: guard bytes around it
+    stay untouched."""
+    p = synth.make_problem(37, 160, 3, "affine", 0.03, "uniform", 8, 3)
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        buf = torch.full((3 * 37 + 64,), 123.0, device="cuda").half()
+        y = buf[32:32 + 3 * 37].view(3, 37)
+        x = to_dev(p.x)
+        h.gemv(x, y)
+        torch.cuda.synchronize()
+        b = buf.cpu()
+        assert torch.all(b[:32] == 123.0) and torch.all(b[32 + 3 * 37:] == 123.0)
+        y_ref, bound = orc.gemv(p)
+        check_y(to_bits(y), y_ref, bound)
+
+
+def test_misaligned_pointers_rejected():
+    p = synth.make_problem(8, 64, 3, "affine", 0.02, "uniform", 1, 1)
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        buf = torch.zeros(200, device="cuda", dtype=torch.float16)
+        rc = dsq.library().dsq_gemv(h._h, buf.data_ptr() + 2, buf.data_ptr() + 256, 1, None)
+        assert rc == dsq.DSQ_ERR_INVALID_ARG
+
+
+def test_streams_and_repeat_calls_agree():
+    p, h = config("c2")
+    x = to_dev(p.x[:1])
+    s = torch.cuda.Stream()
+    y0 = h.gemv(x)
+    with torch.cuda.stream(s):
+        y1 = h.gemv(x, stream=s)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
