@@ -110,7 +110,7 @@ class ClockSampler:
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
                0x2: "applications_clocks_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.002):
+    def __init__(self, index: int, period_s: float = 0.001):
         self.index, self.period = index, period_s
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -295,15 +295,16 @@ def run_dsq(args):
                     call(i)
             graphs.append(g)
     stream.synchronize()
-    for g in graphs:          # one untimed replay of every graph
-        g.replay()
+    with torch.cuda.stream(stream):   # replays launch on the current stream
+        for g in graphs:              # one untimed replay of every graph
+            g.replay()
     stream.synchronize()
 
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     barrier(dist, device)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
+    with ClockSampler(local) as clocks, torch.cuda.stream(stream):
         ev0.record(stream)
         for g in graphs:
             g.replay()
@@ -312,6 +313,8 @@ def run_dsq(args):
     torch.cuda.synchronize()
     barrier(dist, device)
     t_ms = ev0.elapsed_time(ev1)
+    for h in handles:
+        h.check()     # raises if a kernel gave up a bounded wait
     t_max, units = reduce_max_sum(dist, t_ms, canon * K, device)
 
     us_call = t_ms * 1e3 / K
@@ -351,9 +354,10 @@ def run_dsq(args):
                "sample": f"{n} full {args.config} oracle calls at batch {args.batch} "
                          f"({el:.1f} s, single thread)"}
 
+    n_graphs = len(graphs)
+    del graphs
     for h in handles:
         h.close()
-    del graphs
 
     if rank == 0:
         line = {
@@ -369,7 +373,7 @@ def run_dsq(args):
                        "device_bytes_per_call": per_call,
                        "l2": f"rotating {copies} packed copies "
                              f"({copies * per_call / 1e6:.0f} MB > 2x L2 {l2 / 1e6:.0f} MB)",
-                       "timing": f"CUDA events around {len(graphs)} CUDA graph replay(s) "
+                       "timing": f"CUDA events around {n_graphs} CUDA graph replay(s) "
                                  f"of {K} calls"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,

@@ -31,7 +31,7 @@ MODE_LUT_ROW = 0
 MODE_AFFINE_G16 = 1
 
 EXPORTS = ("dsq_pack", "dsq_blob_desc", "dsq_create", "dsq_gemv", "dsq_gemv_launches", "dsq_decode",
-           "dsq_handle_desc", "dsq_device_bytes", "dsq_destroy", "dsq_status_string")
+           "dsq_handle_desc", "dsq_device_bytes", "dsq_check", "dsq_destroy", "dsq_status_string")
 
 
 class DSQError(RuntimeError):
@@ -66,6 +66,7 @@ def library() -> ctypes.CDLL:
         lib.dsq_handle_desc.argtypes = [P, ctypes.POINTER(Desc)]
         lib.dsq_device_bytes.argtypes = [P]
         lib.dsq_device_bytes.restype = SZ
+        lib.dsq_check.argtypes = [P]
         lib.dsq_destroy.argtypes = [P]
         lib.dsq_status_string.argtypes = [I]
         lib.dsq_status_string.restype = ctypes.c_char_p
@@ -208,6 +209,11 @@ class Handle:
                               device=f"cuda:{self.device}")
         _check(library().dsq_decode(self._h, out.data_ptr(), _stream_ptr(stream)), "dsq_decode")
         return out
+
+    def check(self):
+        """Synchronise the device; raise if a kernel of this handle gave up a
+        bounded wait since the last check."""
+        _check(library().dsq_check(self._h), "dsq_check")
 
     def close(self):
         if self._h is not None:

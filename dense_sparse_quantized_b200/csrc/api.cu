@@ -84,8 +84,23 @@ extern "C" int dsq_create(const void *packed, size_t bytes, int device, dsq_hand
     m.dense = (const uint32_t *)(h->d_blob + hd.off_dense);
     m.table = (const uint16_t *)(h->d_blob + hd.off_table);
     m.row_ptr = (const int32_t *)(h->d_blob + hd.off_row_ptr);
-    m.col = (const uint16_t *)(h->d_blob + hd.off_col);
-    m.val = (const uint16_t *)(h->d_blob + hd.off_val);
+    m.csr = (const uint32_t *)(h->d_blob + hd.off_csr);
+    if (cudaMalloc(&h->d_status, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        dsq_destroy(h);
+        return DSQ_ERR_OOM;
+    }
+    h->device_bytes += sizeof(int);
+    if (cudaMemset(h->d_status, 0, sizeof(int)) != cudaSuccess) {
+        dsq_destroy(h);
+        return DSQ_ERR_CUDA;
+    }
+    rc = build_schedule(h, (const int32_t *)((const uint8_t *)packed + hd.off_row_ptr));
+    if (rc == DSQ_OK) rc = fused_prepare(h);
+    if (rc != DSQ_OK) {
+        dsq_destroy(h);
+        return rc;
+    }
     *out = h;
     return DSQ_OK;
 }
@@ -96,12 +111,16 @@ extern "C" int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void 
     if (!aligned16(x) || !aligned16(y)) return DSQ_ERR_INVALID_ARG;
     DeviceGuard guard(h->device);
     if (!guard.ok) return DSQ_ERR_CUDA;
-    return launch_gemv_generic(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
+    int rc = launch_gemv_fused(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
+    if (rc == DSQ_ERR_UNSUPPORTED)
+        rc = launch_gemv_generic(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
+    return rc;
 }
 
 extern "C" int dsq_gemv_launches(dsq_handle_t h, int batch) {
     if (!h || batch < 1) return -1;
-    return gemv_launch_count(h, batch);
+    int n = fused_launch_count(h, batch);
+    return n >= 0 ? n : gemv_launch_count(h, batch);
 }
 
 extern "C" int dsq_decode(dsq_handle_t h, void *w_dense_out, void *stream) {
@@ -128,7 +147,21 @@ extern "C" int dsq_destroy(dsq_handle_t h) {
     DeviceGuard guard(h->device);
     int rc = DSQ_OK;
     if (h->d_blob && cudaFree(h->d_blob) != cudaSuccess) rc = DSQ_ERR_CUDA;
-    if (h->sched.tile_row && cudaFree(h->sched.tile_row) != cudaSuccess) rc = DSQ_ERR_CUDA;
+    if (h->d_status && cudaFree(h->d_status) != cudaSuccess) rc = DSQ_ERR_CUDA;
+    free_schedule(h);
     delete h;
     return rc;
+}
+
+extern "C" int dsq_check(dsq_handle_t h) {
+    if (!h) return DSQ_ERR_INVALID_ARG;
+    DeviceGuard guard(h->device);
+    if (!guard.ok) return DSQ_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return DSQ_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, h->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DSQ_ERR_CUDA;
+    if (word == 0) return DSQ_OK;
+    const int zero = 0;
+    if (cudaMemcpy(h->d_status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return DSQ_ERR_CUDA;
+    return DSQ_ERR_DEVICE;
 }

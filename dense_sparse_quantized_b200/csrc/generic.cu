@@ -74,8 +74,9 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(MatrixView m, const _
     }
     const int k0 = m.row_ptr[row], k1 = m.row_ptr[row + 1];
     for (int k = k0 + lane; k < k1; k += 32) {
-        const float v = __half2float(__ushort_as_half(m.val[k]));
-        const int j = m.col[k];
+        const uint32_t e = __ldg(m.csr + k);
+        const float v = __half2float(__ushort_as_half((unsigned short)(e >> 16)));
+        const int j = (int)(e & 0xffffu);
 #pragma unroll
         for (int b = 0; b < BC; b++)
             if (b < nb) acc[b] = fmaf(v, __half2float(x[(size_t)(b0 + b) * N + j]), acc[b]);

@@ -16,22 +16,35 @@ void plan_blob(const dsq_desc *d, BlobHeader *h);
 int parse_blob(const void *packed, size_t bytes, BlobHeader *out);
 
 // Device view of one packed matrix (pointers into the handle's device copy
-// of the blob) plus the per-device schedule.
+// of the blob).
 struct MatrixView {
     int rows, cols, bits, mode, slots, row_words;
     int64_t nnz;
     const uint32_t *dense;   // rows x row_words
     const uint16_t *table;   // LUT: rows x 2^bits fp16
     const int32_t *row_ptr;  // rows+1
-    const uint16_t *col;     // nnz
-    const uint16_t *val;     // nnz fp16
+    const uint32_t *csr;     // nnz: column | fp16 value << 16
 };
 
-// Row-tile schedule of the batch-1..15 kernels: CTA t owns rows
-// [tile_row[t], tile_row[t+1]).
+// One CTA's share of the batch-1 work: rows [r0, r1), outlier pieces
+// [p0, p1) and the CSR range [k0, k1) those pieces cover.
+struct TileDesc {
+    int32_t r0, r1, p0, p1, k0, k1, pad0, pad1;
+};
+
+// Schedule of the batch-1 kernels, built at create for the device's SM
+// count.  Outliers are cut into "pieces": runs of at most kPieceMax entries
+// of one row; piece p covers CSR entries [piece_k[p], piece_k[p+1]) and row
+// r owns pieces [row_piece[r], row_piece[r+1]).
+constexpr int kPieceMax = 256;
 struct Schedule {
     int n_tiles = 0;
-    int32_t *tile_row = nullptr;  // device, n_tiles+1
+    int max_rows = 0;     // rows of the largest tile
+    int max_pieces = 0;   // pieces of the largest tile
+    int max_csr = 0;      // CSR entries of the largest tile
+    TileDesc *tiles = nullptr;    // device, n_tiles
+    int32_t *row_piece = nullptr; // device, rows+1 (+ padding)
+    int32_t *piece_k = nullptr;   // device, n_pieces+1 (+ padding)
 };
 
 }  // namespace dsq
@@ -44,6 +57,7 @@ struct dsq_handle_s {
     size_t blob_bytes = 0;
     dsq::MatrixView view;
     dsq::Schedule sched;
+    int *d_status = nullptr;  // sticky error word written by kernels on a timed-out wait
     size_t device_bytes = 0;
 };
 
@@ -55,5 +69,13 @@ int launch_gemv_generic(const dsq_handle_s *h, const __half *x, __half *y, int b
 int launch_decode(const dsq_handle_s *h, __half *w, cudaStream_t stream);
 int gemv_launch_count(const dsq_handle_s *h, int batch);
 int launch_zero(__half *y, int64_t n, cudaStream_t stream);
+
+// Tuned batch-1 path (fused_b1.cu).  launch_gemv_fused returns
+// DSQ_ERR_UNSUPPORTED, launching nothing, for shapes it does not cover.
+int build_schedule(dsq_handle_s *h, const int32_t *row_ptr_host);
+void free_schedule(dsq_handle_s *h);
+int fused_prepare(dsq_handle_s *h);
+int fused_launch_count(const dsq_handle_s *h, int batch);
+int launch_gemv_fused(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
 
 }  // namespace dsq

@@ -5,8 +5,8 @@
 //   dense    rows x row_words u32: one "row record" per output row
 //   table    LUT_ROW only: rows x 2^bits fp16 centroids, as given
 //   row_ptr  int32 [rows+1]
-//   col      uint16 [nnz]   CSR column indices (cols <= 65535)
-//   val      fp16   [nnz]   CSR outlier values
+//   csr      uint32 [nnz]   one outlier per word: column index in bits 0..15
+//                           (cols <= 65535), fp16 value in bits 16..31
 //
 // Row record.  The columns of a row are cut into S = ceil(cols/32) "slots"
 // of 32 consecutive columns; the tail slot is padded with code 0 (and, in
@@ -25,13 +25,13 @@
 // scale[2s] | scale[2s+1] << 16 (the two groups of 16 in the slot).
 //
 // Code bits inside a slot.  4-bit: column c in word c/8, bits 4(c%8)..+3.
-// 3-bit: columns are placed so that every field the kernels mask lies in
-// bits 0..22 of a word, or of the word shifted right by 9 -- an fp32 whose
-// exponent field is zero is then the code times 2^-149 exactly (see the
-// kernels).  Column c < 30: word c/10, t = c%10, field at 3t (t < 7) or at
-// 21 + 3(t-7) (t >= 7).  Column 30: bits 0,1 at word 0 bits 30,31 and bit 2
-// at word 1 bit 30.  Column 31: bit 0 at word 1 bit 31, bits 1,2 at word 2
-// bits 30,31.
+// 3-bit: word w (0..2) holds columns 10w..10w+9 as five adjacent pairs; pair
+// j (columns 10w+2j, 10w+2j+1) sits at bits 3j (low half) and 16+3j (high
+// half), so one mask pulls both codes of a pair into the two fp16 halves of
+// a word.  Every field also lies in bits 0..22 of the word, or of the word
+// shifted right by 9, so an AND alone turns it into an exact fp32
+// subnormal.  Columns 30 and 31 use the spare bits: bit k of column 30 is
+// bit 15 of word k, bit k of column 31 is bit 31 of word k.
 #pragma once
 #include <stdint.h>
 
@@ -57,7 +57,7 @@ struct BlobHeader {
     int64_t nnz;
     int32_t slots;      // S
     int32_t row_words;  // u32 words per row record (multiple of 4)
-    uint64_t off_dense, off_table, off_row_ptr, off_col, off_val, total;
+    uint64_t off_dense, off_table, off_row_ptr, off_csr, reserved0, total;
     uint8_t reserved[kHeaderBytes - 8 - 4 - 4 - 16 - 8 - 8 - 48];
 };
 static_assert(sizeof(BlobHeader) == kHeaderBytes, "header size");
@@ -87,19 +87,13 @@ __host__ __device__ inline void code_bit_place(int bits, int c, int k, int *word
         return;
     }
     if (c < 30) {
-        int t = c % 10;
+        const int t = c % 10;
         *word = c / 10;
-        *pos = (t < 7 ? 3 * t : 21 + 3 * (t - 7)) + k;
+        *pos = (t & 1 ? 16 : 0) + 3 * (t >> 1) + k;
         return;
     }
-    if (c == 30) {
-        if (k < 2) { *word = 0; *pos = 30 + k; }
-        else       { *word = 1; *pos = 30; }
-        return;
-    }
-    // c == 31
-    if (k == 0) { *word = 1; *pos = 31; }
-    else        { *word = 2; *pos = 29 + k; }
+    *word = k;
+    *pos = c == 30 ? 15 : 31;
 }
 
 // Word index (inside a record) of code word p of slot s.

@@ -52,10 +52,9 @@ void plan_blob(const dsq_desc *d, BlobHeader *h) {
         off = align_up(off + (uint64_t)d->rows * (1u << d->bits) * 2, kSectionAlign);
     h->off_row_ptr = off;
     off = align_up(off + (uint64_t)(d->rows + 1) * 4, kSectionAlign);
-    h->off_col = off;
-    off = align_up(off + (uint64_t)d->nnz * 2, kSectionAlign);
-    h->off_val = off;
-    off = align_up(off + (uint64_t)d->nnz * 2, kSectionAlign);
+    h->off_csr = off;
+    // +16: kernels copy 16-byte-aligned spans, up to 12 bytes past the end
+    off = align_up(off + (uint64_t)d->nnz * 4 + 16, kSectionAlign);
     h->total = off;
 }
 
@@ -73,8 +72,7 @@ int parse_blob(const void *packed, size_t bytes, BlobHeader *out) {
     plan_blob(&d, &want);
     if (want.slots != h.slots || want.row_words != h.row_words || want.off_dense != h.off_dense ||
         want.off_table != h.off_table || want.off_row_ptr != h.off_row_ptr ||
-        want.off_col != h.off_col || want.off_val != h.off_val || want.total != h.total ||
-        h.total > bytes)
+        want.off_csr != h.off_csr || h.reserved0 != 0 || want.total != h.total || h.total > bytes)
         return DSQ_ERR_INVALID_ARG;
     *out = h;
     return DSQ_OK;
@@ -175,9 +173,8 @@ extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t 
     if (mode == DSQ_MODE_LUT_ROW && M > 0) memcpy(blob + h.off_table, table, (size_t)M * K * 2);
     if (M > 0) memcpy(blob + h.off_row_ptr, row_ptr, (size_t)(M + 1) * 4);
     else memset(blob + h.off_row_ptr, 0, 4);
-    uint16_t *col = (uint16_t *)(blob + h.off_col);
-    for (int64_t k = 0; k < nnz; k++) col[k] = (uint16_t)col_idx[k];
-    if (nnz > 0) memcpy(blob + h.off_val, values, (size_t)nnz * 2);
+    uint32_t *csr = (uint32_t *)(blob + h.off_csr);
+    for (int64_t k = 0; k < nnz; k++) csr[k] = (uint32_t)(uint16_t)col_idx[k] | ((uint32_t)values[k] << 16);
     return DSQ_OK;
 }
 

@@ -166,6 +166,16 @@ DSQ_API int dsq_handle_desc(dsq_handle_t h, dsq_desc *out);
  */
 DSQ_API size_t dsq_device_bytes(dsq_handle_t h);
 
+/*
+ * dsq_check -- synchronise the handle's device and report whether any
+ * kernel launched for this handle gave up a bounded wait (its pipelines
+ * never wait forever: a wait that runs out of iterations abandons the call
+ * and sets a status word).  Returns DSQ_OK, DSQ_ERR_DEVICE (the word was set;
+ * it is cleared, and the y of the affected calls is undefined) or
+ * DSQ_ERR_CUDA.  Host-side; blocks until the device is idle.
+ */
+DSQ_API int dsq_check(dsq_handle_t h);
+
 /* dsq_destroy -- free the handle's device memory; NULL is a no-op.  The
  * caller must make sure no work using the handle is still in flight. */
 DSQ_API int dsq_destroy(dsq_handle_t h);

@@ -159,12 +159,10 @@ def test_empty_shapes_pack():
 def unpack_blob(blob: bytes):
     """Test-only reader of the blob, written from the layout description:
     returns codes, table/scales, zeros, row_ptr, col_idx, values."""
-    b = np.frombuffer(blob, dtype=np.uint8)
-    hdr = np.frombuffer(blob[:96], dtype=np.uint8)
     rows, cols, bits, mode = np.frombuffer(blob[16:32], np.int32)
     nnz = int(np.frombuffer(blob[32:40], np.int64)[0])
     S, row_words = np.frombuffer(blob[40:48], np.int32)
-    off_dense, off_table, off_rp, off_col, off_val, total = np.frombuffer(blob[48:96], np.uint64)
+    off_dense, off_table, off_rp, off_csr, reserved0, total = np.frombuffer(blob[48:96], np.uint64)
     rec = np.frombuffer(blob[int(off_dense):int(off_dense) + rows * row_words * 4],
                         np.uint32).reshape(rows, row_words)
 
@@ -173,15 +171,11 @@ def unpack_blob(blob: bytes):
             return c // 8, 4 * (c % 8) + k
         if c < 30:
             t = c % 10
-            return c // 10, (3 * t if t < 7 else 21 + 3 * (t - 7)) + k
-        if c == 30:
-            return (0, 30 + k) if k < 2 else (1, 30)
-        return (1, 31) if k == 0 else (2, 29 + k)
+            return c // 10, (16 if t % 2 else 0) + 3 * (t // 2) + k
+        return k, (15 if c == 30 else 31)
 
     codes = np.zeros((rows, cols), np.uint8)
     for s in range(S):
-        for p_ in range(bits):
-            pass
         words = [rec[:, (p_ * S + s) if (bits == 3 and mode == 0) else (4 * s + p_)]
                  for p_ in range(bits)]
         for c in range(32):
@@ -211,8 +205,10 @@ def unpack_blob(blob: bytes):
                     table[:, g] = (pair >> np.uint32(16 * e)) & np.uint32(0xFFFF)
                     zeros[:, g] = np.asarray((zb >> (4 * e)) & 15, np.float64).astype(np.float16).view(np.uint16)
     row_ptr = np.frombuffer(blob[int(off_rp):int(off_rp) + (rows + 1) * 4], np.int32)
-    col = np.frombuffer(blob[int(off_col):int(off_col) + nnz * 2], np.uint16).astype(np.int32)
-    val = np.frombuffer(blob[int(off_val):int(off_val) + nnz * 2], np.uint16)
+    csr = np.frombuffer(blob[int(off_csr):int(off_csr) + nnz * 4], np.uint32)
+    col = (csr & np.uint32(0xFFFF)).astype(np.int32)
+    val = (csr >> np.uint32(16)).astype(np.uint16)
+    assert reserved0 == 0 and int(off_csr) + nnz * 4 + 12 <= total
     assert total == len(blob)
     return codes, table, zeros, row_ptr, col, val
 
@@ -230,23 +226,24 @@ def test_layout_round_trip(bits, mode, cols):
     assert np.array_equal(va, p.values)
 
 
-def test_three_bit_fields_sit_below_bit_23():
-    """Every 3-bit field is either inside bits 0..22 of its word or inside bits
-    0..22 after a right shift by 9 (the kernels turn a masked field into an
-    exact fp32 subnormal)."""
-    import itertools
-    seen = set()
+def test_three_bit_fields():
+    """3-bit placement: columns 2j and 2j+1 of a word's ten sit 16 bits apart
+    (one mask puts both into the two fp16 halves, each at bit <= 12 of its
+    half); every field lies in bits 0..22 of its word or of the word >> 9 (an
+    AND then yields an exact fp32 subnormal); columns 30/31 fill bits 15/31;
+    the 96 bits are used once each."""
+    place = {}
     for c in range(32):
         for k in range(3):
             if c < 30:
                 t = c % 10
-                pos = (3 * t if t < 7 else 21 + 3 * (t - 7)) + k
-                word = c // 10
-            elif c == 30:
-                word, pos = (0, 30 + k) if k < 2 else (1, 30)
+                place[c, k] = (c // 10, (16 if t % 2 else 0) + 3 * (t // 2) + k)
             else:
-                word, pos = (1, 31) if k == 0 else (2, 29 + k)
-            assert pos <= 22 or 0 <= pos - 9 <= 22
-            assert (word, pos) not in seen
-            seen.add((word, pos))
-    assert len(seen) == 96
+                place[c, k] = (k, 15 if c == 30 else 31)
+    assert len(set(place.values())) == 96
+    for c in range(0, 30, 2):
+        (w0, p0), (w1, p1) = place[c, 0], place[c + 1, 0]
+        assert w0 == w1 and p1 == p0 + 16 and p0 <= 12
+    for c in range(30):
+        p = place[c, 0][1]
+        assert p + 2 <= 22 or (p - 9 >= 0 and p - 9 + 2 <= 22)

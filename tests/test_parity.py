@@ -49,6 +49,7 @@ def gemv(h, x_bits, batch):
     x = to_dev(x_bits[:batch])
     y = h.gemv(x)
     torch.cuda.synchronize()
+    h.check()
     return to_bits(y)
 
 
