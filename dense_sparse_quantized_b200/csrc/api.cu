@@ -95,8 +95,10 @@ extern "C" int dsq_create(const void *packed, size_t bytes, int device, dsq_hand
         dsq_destroy(h);
         return DSQ_ERR_CUDA;
     }
-    rc = build_schedule(h, (const int32_t *)((const uint8_t *)packed + hd.off_row_ptr));
+    const int32_t *rp_host = (const int32_t *)((const uint8_t *)packed + hd.off_row_ptr);
+    rc = build_schedule(h, rp_host);
     if (rc == DSQ_OK) rc = fused_prepare(h);
+    if (rc == DSQ_OK) rc = tc_prepare(h, rp_host, (const uint32_t *)((const uint8_t *)packed + hd.off_csr));
     if (rc != DSQ_OK) {
         dsq_destroy(h);
         return rc;
@@ -111,7 +113,8 @@ extern "C" int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void 
     if (!aligned16(x) || !aligned16(y)) return DSQ_ERR_INVALID_ARG;
     DeviceGuard guard(h->device);
     if (!guard.ok) return DSQ_ERR_CUDA;
-    int rc = launch_gemv_fused(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
+    int rc = launch_gemv_tc(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
+    if (rc == DSQ_ERR_UNSUPPORTED) rc = launch_gemv_fused(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
     if (rc == DSQ_ERR_UNSUPPORTED)
         rc = launch_gemv_generic(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
     return rc;
@@ -119,7 +122,8 @@ extern "C" int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void 
 
 extern "C" int dsq_gemv_launches(dsq_handle_t h, int batch) {
     if (!h || batch < 1) return -1;
-    int n = fused_launch_count(h, batch);
+    int n = tc_launch_count(h, batch);
+    if (n < 0) n = fused_launch_count(h, batch);
     return n >= 0 ? n : gemv_launch_count(h, batch);
 }
 
@@ -149,6 +153,7 @@ extern "C" int dsq_destroy(dsq_handle_t h) {
     if (h->d_blob && cudaFree(h->d_blob) != cudaSuccess) rc = DSQ_ERR_CUDA;
     if (h->d_status && cudaFree(h->d_status) != cudaSuccess) rc = DSQ_ERR_CUDA;
     free_schedule(h);
+    tc_free(h);
     delete h;
     return rc;
 }

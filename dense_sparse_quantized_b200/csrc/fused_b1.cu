@@ -190,9 +190,23 @@ b1_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
         const int cw = cwarp % C, rg = cwarp / C;
         const int s = cw * 32 + lane;
         const bool valid = s < S;
+        // this lane's 32 columns of x, straight from global memory (coalesced
+        // 16-byte loads; chunks past N read as 0), while the ring fills
+        float xv[32];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            uint4 q = make_uint4(0u, 0u, 0u, 0u);
+            if (valid && s * 32 + 8 * k < m.cols) q = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)s * 32) + k);
+            const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int t = 0; t < 4; t++) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&qw[t]));
+                xv[8 * k + 2 * t] = f.x;
+                xv[8 * k + 2 * t + 1] = f.y;
+            }
+        }
         bool ok = mbar_wait(aux, 0);
         if (!ok) report(p.status, kStatusTimeout);
-        const __half *xs = reinterpret_cast<const __half *>(smem + p.off_x);
         float *part = reinterpret_cast<float *>(smem + p.off_part);
         const int n_st = (nrows + p.R - 1) / p.R;
 
@@ -201,7 +215,7 @@ b1_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
             float XA = 0.f, XB = 0.f;
 #pragma unroll
             for (int c = 0; c < 32; c++) {
-                const float v = valid ? __half2float(xs[s * 32 + c]) : 0.f;
+                const float v = xv[c];
                 if (c < 16) XA += v; else XB += v;
                 const int pc = c < 30 ? pos3(c) : (c == 30 ? 15 : 22);
                 xr[c] = v * __uint_as_float((uint32_t)(127 + 111 - pc) << 23);
@@ -252,9 +266,7 @@ b1_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
                 if (lane == 0) mbar_arrive(&empty[slot]);
             }
         } else {
-            float xr[32];
-#pragma unroll
-            for (int c = 0; c < 32; c++) xr[c] = valid ? __half2float(xs[s * 32 + c]) : 0.f;
+            float (&xr)[32] = xv;
             const __half *tab = reinterpret_cast<const __half *>(smem + p.off_table);
             for (int st = 0; ok && st < n_st; st++) {
                 const int slot = st % p.NS;

@@ -1,5 +1,6 @@
 // internal.h -- private declarations shared by the library's translation units.
 #pragma once
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -47,6 +48,16 @@ struct Schedule {
     int32_t *piece_k = nullptr;   // device, n_pieces+1 (+ padding)
 };
 
+// Tensor-core (batch >= 16) plan: TMA maps over the row records and the
+// K split (a thread-block cluster of KS CTAs per 128-row tile).
+struct TcPlan {
+    bool ready = false;
+    int KS = 1, nkb = 0, kb_per_split = 0;
+    int32_t *split_start = nullptr;  // device, KS x rows (KS > 1)
+    alignas(64) CUtensorMap codes_map;
+    alignas(64) CUtensorMap zero_map;
+};
+
 }  // namespace dsq
 
 struct dsq_handle_s {
@@ -57,6 +68,7 @@ struct dsq_handle_s {
     size_t blob_bytes = 0;
     dsq::MatrixView view;
     dsq::Schedule sched;
+    dsq::TcPlan tc;
     int *d_status = nullptr;  // sticky error word written by kernels on a timed-out wait
     size_t device_bytes = 0;
 };
@@ -77,5 +89,12 @@ void free_schedule(dsq_handle_s *h);
 int fused_prepare(dsq_handle_s *h);
 int fused_launch_count(const dsq_handle_s *h, int batch);
 int launch_gemv_fused(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
+
+// Tensor-core path (tc_b16.cu), same convention.
+int tc_prepare(dsq_handle_s *h, const int32_t *row_ptr_host, const uint32_t *csr_host);
+void tc_free(dsq_handle_s *h);
+bool tc_covers(const dsq_handle_s *h, int batch);
+int tc_launch_count(const dsq_handle_s *h, int batch);
+int launch_gemv_tc(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
 
 }  // namespace dsq

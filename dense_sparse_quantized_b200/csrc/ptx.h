@@ -1,15 +1,17 @@
 // ptx.h -- thin wrappers over the sm_100a PTX this library uses: shared-memory
 // mbarriers, 1-D bulk global->shared copies, and bounded waits.
 //
-// No wait here can spin forever: mbar_wait gives up after `limit` polls and
-// returns false, and every caller then records the failure in the handle's
-// status word (dsq_check reports it) and abandons the call.
+// No wait here can spin forever: mbar_wait gives up after kWaitNs of wall
+// time (read from %globaltimer) and returns false, and every caller then
+// records the failure in the handle's status word (dsq_check reports it) and
+// abandons the call.
 #pragma once
 #include <stdint.h>
 
 namespace dsq {
 
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+constexpr uint32_t kSuspendHintNs = 100000;  // per try_wait, while the phase is incomplete
 constexpr int kStatusTimeout = 1;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -40,24 +42,36 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
         : "memory");
 }
 
+// One test of the phase; while it is incomplete the thread may sleep up to
+// the hinted time (it wakes when the phase completes), so waiting warps do
+// not take issue slots from working ones.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
 
-// True once the barrier's phase with this parity has completed; false after
-// `limit` unsuccessful polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = kWaitLimit) {
-    for (uint32_t i = 0; i < limit; i++)
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// True once the barrier's phase with this parity has completed; false when
+// kWaitNs of wall time pass first (then the caller reports and bails out).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; i++) {
         if (mbar_try_wait(bar, parity)) return true;
-    return false;
+        if ((i & 63u) == 0 && global_ns() - t0 > kWaitNs) return false;
+    }
 }
 
 // 1-D bulk copy global -> this CTA's shared memory, completing `bytes`

@@ -1,0 +1,551 @@
+// tc_b16.cu -- batch >= 16: dequantise to fp16, contract on the 5th-gen
+// tensor cores (tcgen05, accumulator in tensor memory), outliers in fp32.
+//
+// At 16+ activation rows the product is a real (skinny) GEMM, so the dense
+// part goes through tcgen05.mma: for every 128-row tile and 64-column
+// K-block the decoded weights W_dense (bit for bit the fp16 values dsq_decode
+// writes) form the A operand and the x tile the B operand.
+//
+// One CTA per (128-row tile, K split); a K split >1 forms a thread-block
+// cluster whose partial tiles are summed over distributed shared memory into
+// the cluster's rank-0 CTA, which writes y once.  Warp roles:
+//   warp 0      producer: per K-block, three 2-D TMA loads -- the codes and
+//               scales of 128 rows x 2 slots, the 16-byte chunk of zero bytes
+//               holding those slots' zeros, and the x tile [NB rows][64 cols]
+//               in the 128-byte-swizzled K-major layout the MMA reads;
+//   warp 1      allocates tensor memory, issues the MMAs (one thread), frees
+//               tensor memory;
+//   warps 2-9   decode: thread (row = 32*(warp%4) + lane, slot half h) turns
+//               its 32 codes into 16 fp16 pairs -- LOP3 places two codes in
+//               the two halves of 1024.0, one HFMA2 gives the exact q - zero,
+//               one HMUL2 rounds scale*(q - zero) once -- and stores them into
+//               tensor memory (tcgen05.st), the A operand of the MMA;
+//   warps 10-13 outliers: thread (row) walks its row's CSR entries that fall
+//               in each K-block and accumulates v * x[b][col] in fp32 from the
+//               staged x tile (exact products);
+// after the loop warps 2-5 read the accumulator rows (tcgen05.ld), add the
+// outlier sums, reduce over the cluster and store y.
+//
+// Every mbarrier wait is bounded (ptx.h); a wait that runs out sets the
+// handle's status word and the CTA abandons the call, still releasing its
+// tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "internal.h"
+#include "ptx.h"
+
+namespace dsq {
+
+namespace {
+
+constexpr int kTM = 128;        // rows per tile (MMA M)
+constexpr int kKB = 64;         // columns per K-block (two slots)
+constexpr int kStages = 6;
+constexpr int kWarps = 14;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTmemCols = 256;  // accumulator at column 0, A stages from column 64
+constexpr int kACol0 = 64;
+constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
+constexpr uint32_t kSentinel = 0xffffffffu;
+
+struct TcParams {
+    int rows, cols, S, nkb, kb_per_split, batch, zoff_bytes;
+    const int32_t *row_ptr;
+    const uint32_t *csr;
+    const int32_t *split_start;  // [KS][rows] first CSR entry at or past the split's first column; null if KS == 1
+    int *status;
+};
+
+// ------------------------------------------------------------ tcgen05 / TMA
+__device__ __forceinline__ void tma2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; i++) v[i] = __uint_as_float(r[i]);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16, one CTA.
+__device__ __forceinline__ void tc_mma(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d),
+        "r"(a), "l"(bdesc), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// K-major operand, 128-byte swizzle, 8-row core groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(const void *p) {
+    const uint64_t a = (smem_u32(p) >> 4) & 0x3fffu;
+    return a | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor: fp16 A and B (K-major), fp32 accumulator, M = 128.
+__host__ __device__ constexpr uint32_t idesc_f16(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t lop_or_and(uint32_t a, uint32_t mask, uint32_t c) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(c));  // (a & mask) | c
+    return r;
+}
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+// 32 codes of one slot (3 code words + scale pair) -> 16 fp16 pairs equal to
+// fp16(scale * (q - zero)) for columns 2P, 2P+1.
+__device__ __forceinline__ void decode_slot_f16(uint4 v, uint32_t zb, uint32_t (&o)[16]) {
+    const uint32_t zA = zb & 15u, zB = (zb >> 4) & 15u;
+    const __half2 nA = __hneg2(u2h((zA | (zA << 16)) | kMagic));  // -(1024 + zA)
+    const __half2 nB = __hneg2(u2h((zB | (zB << 16)) | kMagic));
+    const __half2 c896 = u2h(0x63006300u), c1008 = u2h(0x63e063e0u);
+    const __half2 dA[3] = {nA, __hadd2(nA, c896), __hadd2(nA, c1008)};  // -(1024 * 8^-t + zA)
+    const __half2 dB[3] = {nB, __hadd2(nB, c896), __hadd2(nB, c1008)};
+    const __half2 cs[3] = {u2h(0x3c003c00u), u2h(0x30003000u), u2h(0x24002400u)};  // 1, 1/8, 1/64
+    uint32_t sA, sB;
+    asm("prmt.b32 %0, %1, %1, 0x1010;" : "=r"(sA) : "r"(v.w));
+    asm("prmt.b32 %0, %1, %1, 0x3232;" : "=r"(sB) : "r"(v.w));
+    const uint32_t a[3] = {v.x, v.y, v.z};
+    const uint32_t b[3] = {v.x >> 9, v.y >> 9, v.z >> 9};
+#pragma unroll
+    for (int P = 0; P < 15; P++) {
+        const int w = P / 5, j = P % 5;
+        const int t = j < 3 ? j : j - 3;  // field at bit 3t of each half
+        const uint32_t h = lop_or_and(j < 3 ? a[w] : b[w], 0x00070007u << (3 * t), kMagic);
+        const __half2 qz = __hfma2(u2h(h), cs[t], P < 8 ? dA[t] : dB[t]);
+        o[P] = h2u(__hmul2(qz, u2h(P < 8 ? sA : sB)));
+    }
+    const uint32_t t15 = ((a[0] >> 15) & 0x00010001u) | ((a[1] >> 14) & 0x00020002u) | ((a[2] >> 13) & 0x00040004u);
+    o[15] = h2u(__hmul2(__hadd2(u2h(t15 | kMagic), nB), u2h(sB)));
+}
+
+// Element (row b, column c) of an x tile [NB][64] fp16 stored by TMA with the
+// 128-byte swizzle (16-byte chunk index XOR row % 8 inside 1024-byte atoms).
+__device__ __forceinline__ int sw128_off(int b, int c) {
+    return ((b >> 3) << 10) + ((b & 7) << 7) + ((((c >> 3) ^ (b & 7))) << 4) + ((c & 7) << 1);
+}
+
+struct Smem {
+    uint64_t *full, *afull, *empty, *done;
+    uint32_t *tmem_slot;
+    unsigned char *x, *codes, *zeros;
+    float *obuf, *rbuf;
+};
+
+template <int NB>
+__device__ __forceinline__ Smem carve(unsigned char *base, int KS) {
+    Smem s;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base);
+    s.full = bars;
+    s.afull = bars + kStages;
+    s.empty = bars + 2 * kStages;
+    s.done = bars + 3 * kStages;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 1);
+    s.x = base + 1024;
+    s.codes = s.x + kStages * NB * 128;
+    s.zeros = s.codes + kStages * kTM * 32;
+    s.obuf = reinterpret_cast<float *>(s.zeros + kStages * kTM * 16);
+    s.rbuf = s.obuf + kTM * NB;
+    (void)KS;
+    return s;
+}
+
+template <int NB>
+__host__ __device__ constexpr size_t smem_bytes(int KS) {
+    return 2048 + (size_t)kStages * (NB * 128 + kTM * 32 + kTM * 16) + (size_t)kTM * NB * 4 * KS;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_cluster_f32(const float *local, uint32_t rank, float v) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_zero,
+          const __grid_constant__ CUtensorMap tm_x, TcParams p, int KS, __half *__restrict__ y) {
+    static_assert(NB == 16 || NB == 32 || NB == 48 || NB == 64, "NB");
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 1024-byte alignment for the swizzled x tiles (1 KB of slack is allocated)
+    unsigned char *smem_base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const Smem sm = carve<NB>(smem_base, KS);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = KS > 1 ? (int)cluster_rank() : 0;
+    const int tile = blockIdx.y;
+    const int kb0 = rank * p.kb_per_split;
+    const int nk = max(0, min(p.nkb, kb0 + p.kb_per_split) - kb0);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; i++) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.afull[i], 8);
+            mbar_init(&sm.empty[i], 1 + 4);
+        }
+        mbar_init(sm.done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(sm.tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *sm.tmem_slot;
+    bool ok = true;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nk; i++) {
+                const int s = i % kStages;
+                if (i >= kStages && !mbar_wait(&sm.empty[s], ((i / kStages) - 1) & 1)) {
+                    report(p.status, kStatusTimeout);
+                    break;
+                }
+                const int kb = kb0 + i;
+                mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(kTM * 32 + kTM * 16 + NB * 128));
+                tma2d(sm.codes + s * kTM * 32, &tm_codes, 8 * kb, kTM * tile, &sm.full[s]);
+                tma2d(sm.zeros + s * kTM * 16, &tm_zero, p.zoff_bytes + 16 * (kb >> 3), kTM * tile, &sm.full[s]);
+                tma2d(sm.x + s * NB * 128, &tm_x, kKB * kb, 0, &sm.full[s]);
+                issued = i + 1;
+            }
+            for (int i = max(0, issued - kStages); i < issued; i++)
+                if (!mbar_wait(&sm.full[i % kStages], (i / kStages) & 1)) report(p.status, kStatusTimeout);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f16(NB);
+            int i = 0;
+            for (; i < nk; i++) {
+                const int s = i % kStages;
+                if (!mbar_wait(&sm.afull[s], (i / kStages) & 1)) {
+                    report(p.status, kStatusTimeout);
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t bdesc = sw128_desc(sm.x + s * NB * 128);
+#pragma unroll
+                for (int k = 0; k < 4; k++)
+                    tc_mma(tmem, tmem + kACol0 + 32 * s + 8 * k, bdesc + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
+                tc_commit(&sm.empty[s]);
+            }
+            tc_commit(sm.done);  // fires once every MMA issued above has completed
+        }
+    } else if (warp < 10) {
+        const int q = warp & 3, h = (warp - 2) >> 2;
+        const int r = 32 * q + lane;
+        const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16);
+        for (int i = 0; i < nk; i++) {
+            const int s = i % kStages;
+            if (!mbar_wait(&sm.full[s], (i / kStages) & 1)) {
+                report(p.status, kStatusTimeout);
+                ok = false;
+                break;
+            }
+            const int slot = 2 * (kb0 + i) + h;
+            uint32_t o[16];
+            if (slot < p.S) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(sm.codes + s * kTM * 32 + r * 32 + 16 * h);
+                const uint32_t zb = sm.zeros[s * kTM * 16 + r * 16 + (slot & 15)];
+                decode_slot_f16(v, zb, o);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; k++) o[k] = 0u;
+            }
+            tc_st16(tbase + kACol0 + 32 * s + 16 * h, o);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.afull[s]);
+        }
+    } else {
+        // outliers: thread = row
+        const int r = 32 * (warp & 3) + lane;
+        const int grow = kTM * tile + r;
+        float acc[NB];
+#pragma unroll
+        for (int b = 0; b < NB; b++) acc[b] = 0.f;
+        int k = 0, kend = 0;
+        if (grow < p.rows && nk > 0) {
+            k = p.split_start ? p.split_start[(size_t)rank * p.rows + grow] : p.row_ptr[grow];
+            kend = p.row_ptr[grow + 1];
+        }
+        uint32_t qv[4];
+#pragma unroll
+        for (int t = 0; t < 4; t++) qv[t] = k + t < kend ? __ldg(p.csr + k + t) : kSentinel;
+        for (int i = 0; i < nk; i++) {
+            const int s = i % kStages;
+            if (!mbar_wait(&sm.full[s], (i / kStages) & 1)) {
+                report(p.status, kStatusTimeout);
+                ok = false;
+                break;
+            }
+            const int c0 = kKB * (kb0 + i);
+            const unsigned char *xt = sm.x + s * NB * 128;
+            while ((int)(qv[0] & 0xffffu) < c0 + kKB) {
+                const int cl = (int)(qv[0] & 0xffffu) - c0;
+                const unsigned short vb = (unsigned short)(qv[0] >> 16);
+#pragma unroll
+                for (int b = 0; b < NB; b++) {
+                    const unsigned short xb = *reinterpret_cast<const unsigned short *>(xt + sw128_off(b, cl));
+                    asm("fma.rn.f32.f16 %0, %1, %2, %0;" : "+f"(acc[b]) : "h"(vb), "h"(xb));
+                }
+                qv[0] = qv[1];
+                qv[1] = qv[2];
+                qv[2] = qv[3];
+                k++;
+                qv[3] = k + 3 < kend ? __ldg(p.csr + k + 3) : kSentinel;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[s]);
+        }
+#pragma unroll
+        for (int b = 0; b < NB; b++) sm.obuf[r * NB + b] = acc[b];
+    }
+
+    __syncthreads();
+    // epilogue: warps 2..5 own accumulator lane quarters 2, 3, 0, 1
+    float part[NB];
+    const bool epi = warp >= 2 && warp < 6;
+    const int q = warp & 3;
+    const int r = 32 * q + lane;
+    const int grow = kTM * tile + r;
+    if (epi) {
+        bool have = nk > 0;
+        if (have && !mbar_wait(sm.done, 0)) {
+            report(p.status, kStatusTimeout);
+            have = false;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < NB; c += 16) {
+            float v[16];
+            if (have) tc_ld16(tmem + ((uint32_t)(32 * q) << 16) + c, v);
+#pragma unroll
+            for (int t = 0; t < 16; t++) part[c + t] = (have ? v[t] : 0.f) + sm.obuf[r * NB + c + t];
+        }
+        if (KS > 1 && rank > 0) {
+#pragma unroll
+            for (int b = 0; b < NB; b++) st_cluster_f32(sm.rbuf + ((size_t)(rank - 1) * kTM + r) * NB + b, 0, part[b]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+    if (KS > 1) cluster_sync();
+    if (epi && rank == 0 && grow < p.rows) {
+        for (int j = 0; j < KS - 1; j++)
+#pragma unroll
+            for (int b = 0; b < NB; b++) part[b] += sm.rbuf[((size_t)j * kTM + r) * NB + b];
+#pragma unroll
+        for (int b = 0; b < NB; b++)
+            if (b < p.batch) y[(size_t)b * p.rows + grow] = __float2half_rn(part[b]);
+    }
+    (void)ok;
+}
+
+// ------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t d0, uint64_t d1,
+               uint64_t stride1_bytes, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {d0, d1};
+    const cuuint64_t strides[1] = {stride1_bytes};
+    const cuuint32_t box[2] = {b0, b1};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NB>
+int launch_nb(const dsq_handle_s *h, const TcParams &p, int KS, const CUtensorMap &tx, __half *y, cudaStream_t st) {
+    const size_t smem = smem_bytes<NB>(KS);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(KS, (h->view.rows + kTM - 1) / kTM, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = KS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_kernel<NB>, h->tc.codes_map, h->tc.zero_map, tx, p, KS, y);
+    return e == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+}
+
+template <int NB>
+int set_attr() {
+    return cudaFuncSetAttribute(tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_bytes<NB>(4)) == cudaSuccess
+               ? DSQ_OK
+               : DSQ_ERR_CUDA;
+}
+
+}  // namespace
+
+bool tc_covers(const dsq_handle_s *h, int batch) {
+    const MatrixView &m = h->view;
+    // cols <= 32768 keeps every K-block's end below the sentinel column 0xffff
+    return h->tc.ready && batch >= 16 && m.rows > 0 && m.cols > 0 && m.cols <= 32768 &&
+           m.mode == DSQ_MODE_AFFINE_G16 && m.bits == 3;
+}
+
+int tc_launch_count(const dsq_handle_s *h, int batch) { return tc_covers(h, batch) ? (batch + 63) / 64 : -1; }
+
+// Tensor maps over the packed rows, the K split and the per-split CSR start
+// of every row.  Host-side, at create, with the device current.
+int tc_prepare(dsq_handle_s *h, const int32_t *rp, const uint32_t *csr_host) {
+    const MatrixView &m = h->view;
+    TcPlan &tc = h->tc;
+    tc.ready = false;
+    if (m.rows == 0 || m.cols == 0 || m.mode != DSQ_MODE_AFFINE_G16 || m.bits != 3) return DSQ_OK;
+    const uint64_t row_bytes = (uint64_t)m.row_words * 4;
+    if (!encode_2d(&tc.codes_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, m.dense, m.row_words, m.rows, row_bytes, 8, kTM,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_2d(&tc.zero_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, m.dense, row_bytes, m.rows, row_bytes, 16, kTM,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+        return DSQ_OK;  // no tensor-map support: the CUDA-core path serves every batch
+    const int tiles = (m.rows + kTM - 1) / kTM;
+    const int nkb = (m.slots + 1) / 2;
+    int KS = 1;
+    for (int k = 2; k <= 4; k++)
+        if (tiles * k <= h->sm_count && k <= nkb) KS = k;
+    tc.KS = KS;
+    tc.nkb = nkb;
+    tc.kb_per_split = (nkb + KS - 1) / KS;
+    if (KS > 1) {
+        std::vector<int32_t> starts((size_t)KS * m.rows);
+        for (int s = 0; s < KS; s++) {
+            const int c0 = s * tc.kb_per_split * kKB;
+            for (int r = 0; r < m.rows; r++) {
+                // first entry of row r with column >= c0 (entries sorted by column)
+                int32_t lo = rp[r], hi = rp[r + 1];
+                while (lo < hi) {
+                    const int32_t mid = lo + (hi - lo) / 2;
+                    const uint32_t e = csr_host[mid];
+                    if ((int)(e & 0xffffu) < c0) lo = mid + 1; else hi = mid;
+                }
+                starts[(size_t)s * m.rows + r] = lo;
+            }
+        }
+        if (cudaMalloc(&tc.split_start, starts.size() * 4) != cudaSuccess) {
+            cudaGetLastError();
+            return DSQ_ERR_OOM;
+        }
+        h->device_bytes += starts.size() * 4;
+        if (cudaMemcpy(tc.split_start, starts.data(), starts.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
+            return DSQ_ERR_CUDA;
+    }
+    int rc = set_attr<16>();
+    if (rc == DSQ_OK) rc = set_attr<32>();
+    if (rc == DSQ_OK) rc = set_attr<64>();
+    if (rc != DSQ_OK) return rc;
+    tc.ready = true;
+    return DSQ_OK;
+}
+
+void tc_free(dsq_handle_s *h) {
+    if (h->tc.split_start) cudaFree(h->tc.split_start);
+    h->tc.split_start = nullptr;
+}
+
+int launch_gemv_tc(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t st) {
+    if (!tc_covers(h, batch)) return DSQ_ERR_UNSUPPORTED;
+    const MatrixView &m = h->view;
+    const TcPlan &tc = h->tc;
+    for (int b0 = 0; b0 < batch; b0 += 64) {
+        const int nb = std::min(64, batch - b0);
+        const int NB = nb <= 16 ? 16 : nb <= 32 ? 32 : 64;
+        CUtensorMap tx;
+        if (!encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x + (size_t)b0 * m.cols, m.cols, nb,
+                       (uint64_t)m.cols * 2, kKB, NB, CU_TENSOR_MAP_SWIZZLE_128B))
+            return DSQ_ERR_CUDA;
+        TcParams p;
+        p.rows = m.rows;
+        p.cols = m.cols;
+        p.S = m.slots;
+        p.nkb = tc.nkb;
+        p.kb_per_split = tc.kb_per_split;
+        p.batch = nb;
+        p.zoff_bytes = 16 * m.slots;
+        p.row_ptr = m.row_ptr;
+        p.csr = m.csr;
+        p.split_start = tc.KS > 1 ? tc.split_start : nullptr;
+        p.status = h->d_status;
+        __half *yb = y + (size_t)b0 * m.rows;
+        int rc;
+        if (NB == 16) rc = launch_nb<16>(h, p, tc.KS, tx, yb, st);
+        else if (NB == 32) rc = launch_nb<32>(h, p, tc.KS, tx, yb, st);
+        else rc = launch_nb<64>(h, p, tc.KS, tx, yb, st);
+        if (rc != DSQ_OK) return rc;
+    }
+    return DSQ_OK;
+}
+
+}  // namespace dsq
