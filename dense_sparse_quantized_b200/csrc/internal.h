@@ -48,14 +48,12 @@ struct Schedule {
     int32_t *piece_k = nullptr;   // device, n_pieces+1 (+ padding)
 };
 
-// Tensor-core (batch >= 16) plan: TMA maps over the row records and the
-// K split (a thread-block cluster of KS CTAs per 128-row tile).
+// Tensor-core (batch >= 16) plan: the K split (a thread-block cluster of KS
+// CTAs per 128-row tile) and where each split starts in every CSR row.
 struct TcPlan {
     bool ready = false;
     int KS = 1, nkb = 0, kb_per_split = 0;
     int32_t *split_start = nullptr;  // device, KS x rows (KS > 1)
-    alignas(64) CUtensorMap codes_map;
-    alignas(64) CUtensorMap zero_map;
 };
 
 }  // namespace dsq

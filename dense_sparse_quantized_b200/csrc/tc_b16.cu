@@ -9,20 +9,22 @@
 // One CTA per (128-row tile, K split); a K split >1 forms a thread-block
 // cluster whose partial tiles are summed over distributed shared memory into
 // the cluster's rank-0 CTA, which writes y once.  Warp roles:
-//   warp 0      producer: per K-block, three 2-D TMA loads -- the codes and
-//               scales of 128 rows x 2 slots, the 16-byte chunk of zero bytes
-//               holding those slots' zeros, and the x tile [NB rows][64 cols]
-//               in the 128-byte-swizzled K-major layout the MMA reads;
-//   warp 1      allocates tensor memory, issues the MMAs (one thread), frees
-//               tensor memory;
-//   warps 2-9   decode: thread (row = 32*(warp%4) + lane, slot half h) turns
-//               its 32 codes into 16 fp16 pairs -- LOP3 places two codes in
-//               the two halves of 1024.0, one HFMA2 gives the exact q - zero,
-//               one HMUL2 rounds scale*(q - zero) once -- and stores them into
-//               tensor memory (tcgen05.st), the A operand of the MMA;
-//   warps 10-13 outliers: thread (row) walks its row's CSR entries that fall
-//               in each K-block and accumulates v * x[b][col] in fp32 from the
-//               staged x tile (exact products);
+//   warp 0       x producer: per K-block, a 2-D TMA load of the x tile
+//                [NB rows][64 cols] into the 128-byte-swizzled K-major layout
+//                the MMA reads (a deep ring; x is small and stays in L2);
+//   warp 1       allocates tensor memory, issues the MMAs (one thread), frees
+//                tensor memory;
+//   warps 2-17   decode: warp (quarter q = warp%4, slot half h, K-block
+//                parity kp) streams, for row 32q + lane, the 16-byte slot
+//                records and zero bytes of every second K-block straight from
+//                HBM (4 K-blocks ahead, double-buffered in registers), turns
+//                the 32 codes into 16 fp16 pairs -- LOP3 places two codes in
+//                the two halves of 1024.0, one HFMA2 gives the exact q - zero,
+//                one HMUL2 rounds scale*(q - zero) once -- and stores them into
+//                tensor memory (tcgen05.st) as the MMA's A operand;
+//   warps 18-21  outliers: thread (row) walks its row's CSR entries that fall
+//                in each K-block and accumulates v * x[b][col] in fp32 from the
+//                staged x tile (exact products);
 // after the loop warps 2-5 read the accumulator rows (tcgen05.ld), add the
 // outlier sums, reduce over the cluster and store y.
 //
@@ -44,16 +46,21 @@ namespace {
 
 constexpr int kTM = 128;        // rows per tile (MMA M)
 constexpr int kKB = 64;         // columns per K-block (two slots)
-constexpr int kStages = 6;
-constexpr int kWarps = 14;
+constexpr int kNA = 6;          // A stages in tensor memory
+constexpr int kU = 4;           // K-blocks a decode warp loads ahead
+constexpr int kWarps = 22;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTmemCols = 256;  // accumulator at column 0, A stages from column 64
 constexpr int kACol0 = 64;
 constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
 constexpr uint32_t kSentinel = 0xffffffffu;
 
+template <int NB>
+__host__ __device__ constexpr int x_stages() { return NB <= 32 ? 12 : 8; }
+
 struct TcParams {
-    int rows, cols, S, nkb, kb_per_split, batch, zoff_bytes;
+    int rows, cols, S, row_words, nkb, kb_per_split, batch;
+    const uint32_t *dense;
     const int32_t *row_ptr;
     const uint32_t *csr;
     const int32_t *split_start;  // [KS][rows] first CSR entry at or past the split's first column; null if KS == 1
@@ -162,33 +169,33 @@ __device__ __forceinline__ int sw128_off(int b, int c) {
 }
 
 struct Smem {
-    uint64_t *full, *afull, *empty, *done;
+    uint64_t *afull, *aempty, *xfull, *xempty, *done;
     uint32_t *tmem_slot;
-    unsigned char *x, *codes, *zeros;
+    unsigned char *x;
     float *obuf, *rbuf;
 };
 
 template <int NB>
-__device__ __forceinline__ Smem carve(unsigned char *base, int KS) {
+__device__ __forceinline__ Smem carve(unsigned char *base) {
+    constexpr int NX = x_stages<NB>();
     Smem s;
     uint64_t *bars = reinterpret_cast<uint64_t *>(base);
-    s.full = bars;
-    s.afull = bars + kStages;
-    s.empty = bars + 2 * kStages;
-    s.done = bars + 3 * kStages;
-    s.tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 1);
+    s.afull = bars;
+    s.aempty = bars + kNA;
+    s.xfull = bars + 2 * kNA;
+    s.xempty = bars + 2 * kNA + NX;
+    s.done = bars + 2 * kNA + 2 * NX;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.done + 1);
     s.x = base + 1024;
-    s.codes = s.x + kStages * NB * 128;
-    s.zeros = s.codes + kStages * kTM * 32;
-    s.obuf = reinterpret_cast<float *>(s.zeros + kStages * kTM * 16);
+    s.obuf = reinterpret_cast<float *>(s.x + NX * NB * 128);
     s.rbuf = s.obuf + kTM * NB;
-    (void)KS;
     return s;
 }
 
+// 1 KB alignment slack + barriers + x ring + outlier sums + cluster inbox.
 template <int NB>
 __host__ __device__ constexpr size_t smem_bytes(int KS) {
-    return 2048 + (size_t)kStages * (NB * 128 + kTM * 32 + kTM * 16) + (size_t)kTM * NB * 4 * KS;
+    return 2048 + (size_t)x_stages<NB>() * NB * 128 + (size_t)kTM * NB * 4 * KS;
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -207,13 +214,13 @@ __device__ __forceinline__ void st_cluster_f32(const float *local, uint32_t rank
 
 template <int NB>
 __global__ void __launch_bounds__(kThreads, 1)
-tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_zero,
-          const __grid_constant__ CUtensorMap tm_x, TcParams p, int KS, __half *__restrict__ y) {
-    static_assert(NB == 16 || NB == 32 || NB == 48 || NB == 64, "NB");
+tc_kernel(const __grid_constant__ CUtensorMap tm_x, TcParams p, int KS, __half *__restrict__ y) {
+    static_assert(NB == 16 || NB == 32 || NB == 64, "NB");
+    constexpr int NX = x_stages<NB>();
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled x tiles (1 KB of slack is allocated)
     unsigned char *smem_base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const Smem sm = carve<NB>(smem_base, KS);
+    const Smem sm = carve<NB>(smem_base);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = KS > 1 ? (int)cluster_rank() : 0;
     const int tile = blockIdx.y;
@@ -221,10 +228,13 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ 
     const int nk = max(0, min(p.nkb, kb0 + p.kb_per_split) - kb0);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; i++) {
-            mbar_init(&sm.full[i], 1);
+        for (int i = 0; i < kNA; i++) {
             mbar_init(&sm.afull[i], 8);
-            mbar_init(&sm.empty[i], 1 + 4);
+            mbar_init(&sm.aempty[i], 1);
+        }
+        for (int i = 0; i < NX; i++) {
+            mbar_init(&sm.xfull[i], 1);
+            mbar_init(&sm.xempty[i], 1 + 4);
         }
         mbar_init(sm.done, 1);
         fence_mbar_init();
@@ -239,34 +249,29 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *sm.tmem_slot;
-    bool ok = true;
 
     if (warp == 0) {
         if (lane == 0) {
             int issued = 0;
             for (int i = 0; i < nk; i++) {
-                const int s = i % kStages;
-                if (i >= kStages && !mbar_wait(&sm.empty[s], ((i / kStages) - 1) & 1)) {
+                const int s = i % NX;
+                if (i >= NX && !mbar_wait(&sm.xempty[s], ((i / NX) - 1) & 1)) {
                     report(p.status, kStatusTimeout);
                     break;
                 }
-                const int kb = kb0 + i;
-                mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(kTM * 32 + kTM * 16 + NB * 128));
-                tma2d(sm.codes + s * kTM * 32, &tm_codes, 8 * kb, kTM * tile, &sm.full[s]);
-                tma2d(sm.zeros + s * kTM * 16, &tm_zero, p.zoff_bytes + 16 * (kb >> 3), kTM * tile, &sm.full[s]);
-                tma2d(sm.x + s * NB * 128, &tm_x, kKB * kb, 0, &sm.full[s]);
+                mbar_arrive_expect_tx(&sm.xfull[s], (uint32_t)(NB * 128));
+                tma2d(sm.x + s * NB * 128, &tm_x, kKB * (kb0 + i), 0, &sm.xfull[s]);
                 issued = i + 1;
             }
-            for (int i = max(0, issued - kStages); i < issued; i++)
-                if (!mbar_wait(&sm.full[i % kStages], (i / kStages) & 1)) report(p.status, kStatusTimeout);
+            for (int i = max(0, issued - NX); i < issued; i++)
+                if (!mbar_wait(&sm.xfull[i % NX], (i / NX) & 1)) report(p.status, kStatusTimeout);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = idesc_f16(NB);
-            int i = 0;
-            for (; i < nk; i++) {
-                const int s = i % kStages;
-                if (!mbar_wait(&sm.afull[s], (i / kStages) & 1)) {
+            for (int i = 0; i < nk; i++) {
+                const int a = i % kNA, s = i % NX;
+                if (!mbar_wait(&sm.afull[a], (i / kNA) & 1) || !mbar_wait(&sm.xfull[s], (i / NX) & 1)) {
                     report(p.status, kStatusTimeout);
                     break;
                 }
@@ -274,37 +279,63 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ 
                 const uint64_t bdesc = sw128_desc(sm.x + s * NB * 128);
 #pragma unroll
                 for (int k = 0; k < 4; k++)
-                    tc_mma(tmem, tmem + kACol0 + 32 * s + 8 * k, bdesc + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
-                tc_commit(&sm.empty[s]);
+                    tc_mma(tmem, tmem + kACol0 + 32 * a + 8 * k, bdesc + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
+                tc_commit(&sm.aempty[a]);
+                tc_commit(&sm.xempty[s]);
             }
             tc_commit(sm.done);  // fires once every MMA issued above has completed
         }
-    } else if (warp < 10) {
-        const int q = warp & 3, h = (warp - 2) >> 2;
+    } else if (warp < 18) {
+        const int d = warp - 2;
+        const int q = warp & 3, h = (d >> 2) & 1, kp = d >> 3;
         const int r = 32 * q + lane;
+        const int grow = kTM * tile + r;
         const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16);
-        for (int i = 0; i < nk; i++) {
-            const int s = i % kStages;
-            if (!mbar_wait(&sm.full[s], (i / kStages) & 1)) {
-                report(p.status, kStatusTimeout);
-                ok = false;
-                break;
-            }
-            const int slot = 2 * (kb0 + i) + h;
-            uint32_t o[16];
-            if (slot < p.S) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(sm.codes + s * kTM * 32 + r * 32 + 16 * h);
-                const uint32_t zb = sm.zeros[s * kTM * 16 + r * 16 + (slot & 15)];
-                decode_slot_f16(v, zb, o);
-            } else {
+        const uint32_t *rec = p.dense + (size_t)min(grow, p.rows - 1) * p.row_words;
+        uint4 cur[kU], nxt[kU];
+        uint32_t czb[kU], nzb[kU];
+        // K-blocks of this warp: kp, kp + 2, ...; batch j holds the kU K-blocks kp + 2*(kU*j + u)
+        auto load = [&](int j, uint4 (&v)[kU], uint32_t (&zb)[kU]) {
 #pragma unroll
-                for (int k = 0; k < 16; k++) o[k] = 0u;
+            for (int u = 0; u < kU; u++) {
+                const int i = kp + 2 * (kU * j + u);
+                const int slot = 2 * (kb0 + i) + h;
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+                zb[u] = 0u;
+                if (i < nk && slot < p.S && grow < p.rows) {
+                    v[u] = __ldg(reinterpret_cast<const uint4 *>(rec) + slot);
+                    zb[u] = __ldg(reinterpret_cast<const uint8_t *>(rec + 4 * p.S) + slot);
+                }
             }
-            tc_st16(tbase + kACol0 + 32 * s + 16 * h, o);
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.afull[s]);
+        };
+        load(0, cur, czb);
+        bool ok = true;
+        for (int j = 0; ok && kp + 2 * kU * j < nk; j++) {
+            load(j + 1, nxt, nzb);
+#pragma unroll
+            for (int u = 0; u < kU; u++) {
+                const int i = kp + 2 * (kU * j + u);
+                if (i >= nk) break;  // warp-uniform
+                const int a = i % kNA;
+                if (i >= kNA && !mbar_wait_warp(&sm.aempty[a], ((i / kNA) - 1) & 1)) {
+                    if (lane == 0) report(p.status, kStatusTimeout);
+                    ok = false;
+                    break;
+                }
+                uint32_t o[16];
+                decode_slot_f16(cur[u], czb[u], o);  // zero records decode to 0 (scale 0)
+                tc_fence_after();
+                tc_st16(tbase + kACol0 + 32 * a + 16 * h, o);
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.afull[a]);
+            }
+#pragma unroll
+            for (int u = 0; u < kU; u++) {
+                cur[u] = nxt[u];
+                czb[u] = nzb[u];
+            }
         }
     } else {
         // outliers: thread = row
@@ -322,10 +353,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ 
 #pragma unroll
         for (int t = 0; t < 4; t++) qv[t] = k + t < kend ? __ldg(p.csr + k + t) : kSentinel;
         for (int i = 0; i < nk; i++) {
-            const int s = i % kStages;
-            if (!mbar_wait(&sm.full[s], (i / kStages) & 1)) {
-                report(p.status, kStatusTimeout);
-                ok = false;
+            const int s = i % NX;
+            if (!mbar_wait_warp(&sm.xfull[s], (i / NX) & 1)) {
+                if (lane == 0) report(p.status, kStatusTimeout);
                 break;
             }
             const int c0 = kKB * (kb0 + i);
@@ -345,7 +375,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ 
                 qv[3] = k + 3 < kend ? __ldg(p.csr + k + 3) : kSentinel;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty[s]);
+            if (lane == 0) mbar_arrive(&sm.xempty[s]);
         }
 #pragma unroll
         for (int b = 0; b < NB; b++) sm.obuf[r * NB + b] = acc[b];
@@ -360,8 +390,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ 
     const int grow = kTM * tile + r;
     if (epi) {
         bool have = nk > 0;
-        if (have && !mbar_wait(sm.done, 0)) {
-            report(p.status, kStatusTimeout);
+        if (have && !mbar_wait_warp(sm.done, 0)) {
+            if (lane == 0) report(p.status, kStatusTimeout);
             have = false;
         }
         tc_fence_after();
@@ -392,7 +422,6 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ 
         for (int b = 0; b < NB; b++)
             if (b < p.batch) y[(size_t)b * p.rows + grow] = __float2half_rn(part[b]);
     }
-    (void)ok;
 }
 
 // ------------------------------------------------------------ host side
@@ -421,12 +450,11 @@ bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_
 }
 
 template <int NB>
-int launch_nb(const dsq_handle_s *h, const TcParams &p, int KS, const CUtensorMap &tx, __half *y, cudaStream_t st) {
-    const size_t smem = smem_bytes<NB>(KS);
+int launch_nb(const TcParams &p, int KS, const CUtensorMap &tx, __half *y, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(KS, (h->view.rows + kTM - 1) / kTM, 1);
+    cfg.gridDim = dim3(KS, (p.rows + kTM - 1) / kTM, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = smem_bytes<NB>(KS);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -435,8 +463,7 @@ int launch_nb(const dsq_handle_s *h, const TcParams &p, int KS, const CUtensorMa
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_kernel<NB>, h->tc.codes_map, h->tc.zero_map, tx, p, KS, y);
-    return e == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, tc_kernel<NB>, tx, p, KS, y) == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
 }
 
 template <int NB>
@@ -447,38 +474,86 @@ int set_attr() {
                : DSQ_ERR_CUDA;
 }
 
+int set_attrs() {
+    int rc = set_attr<16>();
+    if (rc == DSQ_OK) rc = set_attr<32>();
+    if (rc == DSQ_OK) rc = set_attr<64>();
+    return rc;
+}
+
+// K split of a matrix: KS CTAs (one cluster) per 128-row tile, as many as fit
+// one CTA per SM, at most 4 and at most one per K-block.
+struct Split {
+    int KS, nkb, kb_per_split;
+};
+Split plan_split(const MatrixView &m, int sm_count) {
+    Split sp;
+    const int tiles = (m.rows + kTM - 1) / kTM;
+    sp.nkb = (m.slots + 1) / 2;
+    sp.KS = 1;
+    for (int k = 2; k <= 4; k++)
+        if (tiles * k <= sm_count && k <= sp.nkb) sp.KS = k;
+    sp.kb_per_split = (sp.nkb + sp.KS - 1) / sp.KS;
+    return sp;
+}
+
+bool tc_shape_ok(const MatrixView &m) {
+    // cols <= 32768 keeps every K-block's end below the sentinel column 0xffff
+    return m.rows > 0 && m.cols > 0 && m.cols <= 32768 && m.mode == DSQ_MODE_AFFINE_G16 && m.bits == 3;
+}
+
+// All launches of one product (batch in chunks of 64 rows of x).
+int run_tc(const MatrixView &m, const Split &sp, const int32_t *split_start, int *status, const __half *x,
+           __half *y, int batch, cudaStream_t st) {
+    for (int b0 = 0; b0 < batch; b0 += 64) {
+        const int nb = std::min(64, batch - b0);
+        const int NB = nb <= 16 ? 16 : nb <= 32 ? 32 : 64;
+        CUtensorMap tx;
+        if (!encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x + (size_t)b0 * m.cols, m.cols, nb,
+                       (uint64_t)m.cols * 2, kKB, NB, CU_TENSOR_MAP_SWIZZLE_128B))
+            return DSQ_ERR_CUDA;
+        TcParams p;
+        p.rows = m.rows;
+        p.cols = m.cols;
+        p.S = m.slots;
+        p.row_words = m.row_words;
+        p.nkb = sp.nkb;
+        p.kb_per_split = sp.kb_per_split;
+        p.batch = nb;
+        p.dense = m.dense;
+        p.row_ptr = m.row_ptr;
+        p.csr = m.csr;
+        p.split_start = sp.KS > 1 ? split_start : nullptr;
+        p.status = status;
+        __half *yb = y + (size_t)b0 * m.rows;
+        int rc;
+        if (NB == 16) rc = launch_nb<16>(p, sp.KS, tx, yb, st);
+        else if (NB == 32) rc = launch_nb<32>(p, sp.KS, tx, yb, st);
+        else rc = launch_nb<64>(p, sp.KS, tx, yb, st);
+        if (rc != DSQ_OK) return rc;
+    }
+    return DSQ_OK;
+}
+
 }  // namespace
 
-bool tc_covers(const dsq_handle_s *h, int batch) {
-    const MatrixView &m = h->view;
-    // cols <= 32768 keeps every K-block's end below the sentinel column 0xffff
-    return h->tc.ready && batch >= 16 && m.rows > 0 && m.cols > 0 && m.cols <= 32768 &&
-           m.mode == DSQ_MODE_AFFINE_G16 && m.bits == 3;
-}
+bool tc_covers(const dsq_handle_s *h, int batch) { return h->tc.ready && batch >= 16 && tc_shape_ok(h->view); }
 
 int tc_launch_count(const dsq_handle_s *h, int batch) { return tc_covers(h, batch) ? (batch + 63) / 64 : -1; }
 
-// Tensor maps over the packed rows, the K split and the per-split CSR start
-// of every row.  Host-side, at create, with the device current.
+// K split and the per-split CSR start of every row.  Host-side, at create,
+// with the device current.
 int tc_prepare(dsq_handle_s *h, const int32_t *rp, const uint32_t *csr_host) {
     const MatrixView &m = h->view;
     TcPlan &tc = h->tc;
     tc.ready = false;
-    if (m.rows == 0 || m.cols == 0 || m.mode != DSQ_MODE_AFFINE_G16 || m.bits != 3) return DSQ_OK;
-    const uint64_t row_bytes = (uint64_t)m.row_words * 4;
-    if (!encode_2d(&tc.codes_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, m.dense, m.row_words, m.rows, row_bytes, 8, kTM,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_2d(&tc.zero_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, m.dense, row_bytes, m.rows, row_bytes, 16, kTM,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
-        return DSQ_OK;  // no tensor-map support: the CUDA-core path serves every batch
-    const int tiles = (m.rows + kTM - 1) / kTM;
-    const int nkb = (m.slots + 1) / 2;
-    int KS = 1;
-    for (int k = 2; k <= 4; k++)
-        if (tiles * k <= h->sm_count && k <= nkb) KS = k;
+    if (!tc_shape_ok(m)) return DSQ_OK;
+    if (!encode_fn()) return DSQ_OK;  // no tensor-map support: the CUDA-core path serves every batch
+    const Split sp = plan_split(m, h->sm_count);
+    const int KS = sp.KS;
     tc.KS = KS;
-    tc.nkb = nkb;
-    tc.kb_per_split = (nkb + KS - 1) / KS;
+    tc.nkb = sp.nkb;
+    tc.kb_per_split = sp.kb_per_split;
     if (KS > 1) {
         std::vector<int32_t> starts((size_t)KS * m.rows);
         for (int s = 0; s < KS; s++) {
@@ -488,8 +563,7 @@ int tc_prepare(dsq_handle_s *h, const int32_t *rp, const uint32_t *csr_host) {
                 int32_t lo = rp[r], hi = rp[r + 1];
                 while (lo < hi) {
                     const int32_t mid = lo + (hi - lo) / 2;
-                    const uint32_t e = csr_host[mid];
-                    if ((int)(e & 0xffffu) < c0) lo = mid + 1; else hi = mid;
+                    if ((int)(csr_host[mid] & 0xffffu) < c0) lo = mid + 1; else hi = mid;
                 }
                 starts[(size_t)s * m.rows + r] = lo;
             }
@@ -502,9 +576,7 @@ int tc_prepare(dsq_handle_s *h, const int32_t *rp, const uint32_t *csr_host) {
         if (cudaMemcpy(tc.split_start, starts.data(), starts.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
             return DSQ_ERR_CUDA;
     }
-    int rc = set_attr<16>();
-    if (rc == DSQ_OK) rc = set_attr<32>();
-    if (rc == DSQ_OK) rc = set_attr<64>();
+    const int rc = set_attrs();
     if (rc != DSQ_OK) return rc;
     tc.ready = true;
     return DSQ_OK;
@@ -517,35 +589,9 @@ void tc_free(dsq_handle_s *h) {
 
 int launch_gemv_tc(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t st) {
     if (!tc_covers(h, batch)) return DSQ_ERR_UNSUPPORTED;
-    const MatrixView &m = h->view;
-    const TcPlan &tc = h->tc;
-    for (int b0 = 0; b0 < batch; b0 += 64) {
-        const int nb = std::min(64, batch - b0);
-        const int NB = nb <= 16 ? 16 : nb <= 32 ? 32 : 64;
-        CUtensorMap tx;
-        if (!encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x + (size_t)b0 * m.cols, m.cols, nb,
-                       (uint64_t)m.cols * 2, kKB, NB, CU_TENSOR_MAP_SWIZZLE_128B))
-            return DSQ_ERR_CUDA;
-        TcParams p;
-        p.rows = m.rows;
-        p.cols = m.cols;
-        p.S = m.slots;
-        p.nkb = tc.nkb;
-        p.kb_per_split = tc.kb_per_split;
-        p.batch = nb;
-        p.zoff_bytes = 16 * m.slots;
-        p.row_ptr = m.row_ptr;
-        p.csr = m.csr;
-        p.split_start = tc.KS > 1 ? tc.split_start : nullptr;
-        p.status = h->d_status;
-        __half *yb = y + (size_t)b0 * m.rows;
-        int rc;
-        if (NB == 16) rc = launch_nb<16>(h, p, tc.KS, tx, yb, st);
-        else if (NB == 32) rc = launch_nb<32>(h, p, tc.KS, tx, yb, st);
-        else rc = launch_nb<64>(h, p, tc.KS, tx, yb, st);
-        if (rc != DSQ_OK) return rc;
-    }
-    return DSQ_OK;
+    const Split sp = {h->tc.KS, h->tc.nkb, h->tc.kb_per_split};
+    return run_tc(h->view, sp, h->tc.split_start, h->d_status, x, y, batch, st);
 }
 
 }  // namespace dsq
+
