@@ -27,11 +27,13 @@ DSQ_ERR_CUDA = -3
 DSQ_ERR_OOM = -4
 DSQ_ERR_BUFFER_TOO_SMALL = -5
 DSQ_ERR_DEVICE = -6
+DSQ_ERR_SCRATCH_LIMIT = -7
 MODE_LUT_ROW = 0
 MODE_AFFINE_G16 = 1
 
 EXPORTS = ("dsq_pack", "dsq_blob_desc", "dsq_create", "dsq_gemv", "dsq_gemv_launches", "dsq_decode",
-           "dsq_handle_desc", "dsq_device_bytes", "dsq_check", "dsq_destroy", "dsq_status_string")
+           "dsq_handle_desc", "dsq_device_bytes", "dsq_check", "dsq_destroy", "dsq_status_string",
+           "dsq_gemv_noalloc")
 
 
 class DSQError(RuntimeError):
@@ -68,6 +70,7 @@ def library() -> ctypes.CDLL:
         lib.dsq_device_bytes.restype = SZ
         lib.dsq_check.argtypes = [P]
         lib.dsq_destroy.argtypes = [P]
+        lib.dsq_gemv_noalloc.argtypes = [ctypes.POINTER(Desc), P, SZ, P, P, I, P]
         lib.dsq_status_string.argtypes = [I]
         lib.dsq_status_string.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -231,3 +234,26 @@ class Handle:
 
     def __exit__(self, *exc):
         self.close()
+
+
+def gemv_noalloc(desc: Desc, packed_device, x, y, stream=None):
+    """y = x @ What^T without a handle and without any device allocation in
+    the library, for callers whose device memory all comes from a host
+    program's own pool.  ``packed_device``: the dsq_pack blob already copied
+    to the device by the caller (a cuda uint8 tensor, 256-byte aligned);
+    ``x``: cuda fp16 [batch, cols]; ``y``: caller-allocated cuda fp16
+    [batch, rows].  Calls that overlap on the GPU share one scratch array and
+    race.  Asynchronous on ``stream`` (default: the current torch stream)."""
+    import torch
+    if packed_device.dtype != torch.uint8 or not packed_device.is_cuda or not packed_device.is_contiguous():
+        raise ValueError("packed_device must be a contiguous cuda uint8 tensor")
+    for name, t in (("x", x), ("y", y)):
+        if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 2:
+            raise ValueError(f"{name} must be a contiguous 2-D cuda float16 tensor")
+    batch = x.shape[0]
+    if x.shape[1] != desc.cols or tuple(y.shape) != (batch, desc.rows):
+        raise ValueError("x must be [batch, cols] and y [batch, rows]")
+    _check(library().dsq_gemv_noalloc(ctypes.byref(desc), packed_device.data_ptr(), packed_device.numel(),
+                                      x.data_ptr(), y.data_ptr(), batch, _stream_ptr(stream)),
+           "dsq_gemv_noalloc")
+    return y

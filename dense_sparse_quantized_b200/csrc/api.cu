@@ -38,6 +38,8 @@ extern "C" const char *dsq_status_string(int status) {
         case DSQ_ERR_OOM: return "DSQ_ERR_OOM: device allocation failed";
         case DSQ_ERR_BUFFER_TOO_SMALL: return "DSQ_ERR_BUFFER_TOO_SMALL: output buffer too small";
         case DSQ_ERR_DEVICE: return "DSQ_ERR_DEVICE: a kernel reported an error";
+        case DSQ_ERR_SCRATCH_LIMIT:
+            return "DSQ_ERR_SCRATCH_LIMIT: the matrix needs more than dsq_gemv_noalloc's fixed scratch";
         default: return "unknown dsq status";
     }
 }

@@ -35,6 +35,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "internal.h"
@@ -595,3 +596,126 @@ int launch_gemv_tc(const dsq_handle_s *h, const __half *x, __half *y, int batch,
 
 }  // namespace dsq
 
+// ---------------------------------------------------------------------------
+// dsq_gemv_noalloc: the tensor-core product for callers that cannot allocate
+// device memory.  The only memory the kernels need besides the caller's
+// buffers -- the status word and the per-split CSR starts -- lives in one
+// fixed array that every GPU loading this library holds until exit.
+// ---------------------------------------------------------------------------
+
+namespace dsq {
+
+namespace {
+
+// 256 KiB: word 0 is the status word, words [kNoAllocStartsOff, ...) the
+// split starts ([KS][rows], KS > 1 only).
+constexpr int kNoAllocWords = 65536;
+constexpr int kNoAllocStartsOff = 64;
+constexpr int kNoAllocMaxStarts = kNoAllocWords - kNoAllocStartsOff;
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocWords];
+
+// Clears the status word and, for a K split, finds in every row the first CSR
+// entry at or past each split's first column (entries sorted by column).
+__global__ void noalloc_prep_kernel(int32_t *scratch, const int32_t *row_ptr, const uint32_t *csr, int rows,
+                                    int KS, int cols_per_split) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i == 0) scratch[0] = 0;
+    if (KS <= 1 || i >= (int64_t)KS * rows) return;
+    const int s = (int)(i / rows), r = (int)(i % rows);
+    const int c0 = s * cols_per_split;
+    int32_t lo = row_ptr[r], hi = row_ptr[r + 1];
+    while (lo < hi) {
+        const int32_t mid = lo + (hi - lo) / 2;
+        if ((int)(csr[mid] & 0xffffu) < c0) lo = mid + 1; else hi = mid;
+    }
+    scratch[kNoAllocStartsOff + i] = lo;
+}
+
+struct NoAllocDevice {
+    bool ready = false;
+    int sm_count = 0;
+    int32_t *scratch = nullptr;  // device address of g_noalloc_scratch on this device
+};
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+
+// Once per device, with that device current: check the architecture, look up
+// the scratch array's device address and set the kernels' shared-memory limit.
+int noalloc_setup(int dev, NoAllocDevice *out) {
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return DSQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoAllocDevice &d = g_noalloc_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return DSQ_ERR_CUDA;
+        if (major != 10 || minor != 0 || !encode_fn()) return DSQ_ERR_UNSUPPORTED;
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+            cudaGetLastError();
+            return DSQ_ERR_CUDA;
+        }
+        const int rc = set_attrs();
+        if (rc != DSQ_OK) return rc;
+        d.sm_count = sms;
+        d.scratch = (int32_t *)ptr;
+        d.ready = true;
+    }
+    *out = d;
+    return DSQ_OK;
+}
+
+}  // namespace
+
+}  // namespace dsq
+
+extern "C" int dsq_gemv_noalloc(const dsq_desc *d, const void *packed_device, size_t bytes, const void *x, void *y,
+                                int batch, void *stream) {
+    using namespace dsq;
+    if (!d || batch < 1) return DSQ_ERR_INVALID_ARG;
+    int rc = check_desc(d);
+    if (rc != DSQ_OK) return rc;
+    BlobHeader hd;
+    plan_blob(d, &hd);
+    if (bytes != hd.total) return DSQ_ERR_INVALID_ARG;
+    if (d->rows == 0) return DSQ_OK;
+    if (!packed_device || ((uintptr_t)packed_device & 255u) || !y || ((uintptr_t)y & 15u) ||
+        (d->cols > 0 && (!x || ((uintptr_t)x & 15u))))
+        return DSQ_ERR_INVALID_ARG;
+    if (d->mode != DSQ_MODE_AFFINE_G16 || d->bits != 3 || d->cols > 32768 || batch < 16) return DSQ_ERR_UNSUPPORTED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DSQ_ERR_CUDA;
+    NoAllocDevice nd;
+    rc = noalloc_setup(dev, &nd);
+    if (rc != DSQ_OK) return rc;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (d->cols == 0) return launch_zero((__half *)y, (int64_t)batch * d->rows, st);
+
+    const uint8_t *base = (const uint8_t *)packed_device;
+    MatrixView m;
+    m.rows = hd.rows;
+    m.cols = hd.cols;
+    m.bits = hd.bits;
+    m.mode = hd.mode;
+    m.slots = hd.slots;
+    m.row_words = hd.row_words;
+    m.nnz = hd.nnz;
+    m.dense = (const uint32_t *)(base + hd.off_dense);
+    m.table = (const uint16_t *)(base + hd.off_table);
+    m.row_ptr = (const int32_t *)(base + hd.off_row_ptr);
+    m.csr = (const uint32_t *)(base + hd.off_csr);
+    const Split sp = plan_split(m, nd.sm_count);
+    const int64_t starts = sp.KS > 1 ? (int64_t)sp.KS * m.rows : 0;
+    if (starts > kNoAllocMaxStarts) return DSQ_ERR_SCRATCH_LIMIT;
+
+    const int64_t n_prep = std::max<int64_t>(1, starts);
+    noalloc_prep_kernel<<<(unsigned)((n_prep + 255) / 256), 256, 0, st>>>(
+        nd.scratch, m.row_ptr, m.csr, m.rows, sp.KS, sp.kb_per_split * kKB);
+    if (cudaGetLastError() != cudaSuccess) return DSQ_ERR_CUDA;
+    return run_tc(m, sp, nd.scratch + kNoAllocStartsOff, (int *)nd.scratch, (const __half *)x, (__half *)y, batch,
+                  st);
+}

@@ -56,7 +56,8 @@ typedef enum {
     DSQ_ERR_CUDA = -3,            /* a CUDA runtime call or a kernel launch failed */
     DSQ_ERR_OOM = -4,             /* device allocation failed */
     DSQ_ERR_BUFFER_TOO_SMALL = -5,/* output buffer smaller than required; size reported */
-    DSQ_ERR_DEVICE = -6           /* a kernel reported an error through its status word */
+    DSQ_ERR_DEVICE = -6,          /* a kernel reported an error through its status word */
+    DSQ_ERR_SCRATCH_LIMIT = -7    /* dsq_gemv_noalloc: the problem needs more than its fixed scratch */
 } dsq_status;
 
 enum { DSQ_MODE_LUT_ROW = 0, DSQ_MODE_AFFINE_G16 = 1 };
@@ -179,6 +180,56 @@ DSQ_API int dsq_check(dsq_handle_t h);
 /* dsq_destroy -- free the handle's device memory; NULL is a no-op.  The
  * caller must make sure no work using the handle is still in flight. */
 DSQ_API int dsq_destroy(dsq_handle_t h);
+
+/*
+ * dsq_gemv_noalloc -- the product of dsq_gemv for a caller that may not
+ * allocate device memory: y[b][i] = sum_j x[b][j] * What[i][j], b < batch.
+ * The paper has no counterpart; this entry point exists for integration.
+ *
+ * Who needs it: code whose device memory all belongs to a host program --
+ * a plugin that runs inside an inference engine or framework that hands out
+ * every device buffer from its own pool (a cudaMalloc there would fragment
+ * or escape the pool, or be forbidden outright), and code that runs where
+ * cudaMalloc's implicit device synchronisation is not allowed.  Such a caller
+ * cannot create a handle (dsq_create allocates), so it uploads the blob from
+ * dsq_pack into memory it owns and calls this function with no handle.
+ *
+ * d             host; the blob's shape (as dsq_blob_desc reports it).
+ * packed_device device; the dsq_pack blob copied verbatim, `bytes` long
+ *               (exactly the size dsq_pack reported), 256-byte aligned.
+ *               Read only; the caller owns it.
+ * x, y, batch, stream  as for dsq_gemv (fp16 [batch][cols] / [batch][rows],
+ *               16-byte aligned, on the current device).
+ *
+ * Covers what the tensor-core path covers: 3-bit affine (DSQ_MODE_AFFINE_G16)
+ * matrices with cols <= 32768 and batch >= 16; anything else returns
+ * DSQ_ERR_UNSUPPORTED and launches nothing.  Results equal dsq_gemv's for the
+ * same inputs on the same device.
+ *
+ * Memory: no device allocation of any kind.  The scratch the kernels need
+ * (a status word and the start of every CSR row in each K split) is one
+ * fixed 256 KiB array of the library that every GPU which loads it holds
+ * until the process exits.  At most 65472 split-start entries fit: a
+ * matrix whose K split needs more (split count x rows) is refused with
+ * DSQ_ERR_SCRATCH_LIMIT before any launch.  Each call first clears the
+ * status word and rewrites the split starts, so nothing of an earlier call
+ * leaks into it; but every call on a device shares that one array, so calls
+ * whose kernels overlap on the GPU (other streams, other host threads) race
+ * and give undefined y: order them on one stream or with events.
+ *
+ * The first call on each device, with that device current, does a one-time
+ * set-up (looks up the array's device address, sets the kernels' shared-
+ * memory limit); make that first call before any stream capture.  A bounded
+ * wait that runs out inside the kernels (a broken device, never a normal
+ * call) leaves y of that call undefined; this entry point has no status
+ * read-back.
+ *
+ * Returns DSQ_OK, DSQ_ERR_INVALID_ARG (NULL or misaligned pointer, batch <
+ * 1, bytes not the blob's size, malformed desc), DSQ_ERR_UNSUPPORTED,
+ * DSQ_ERR_SCRATCH_LIMIT or DSQ_ERR_CUDA.  Asynchronous on `stream`.
+ */
+DSQ_API int dsq_gemv_noalloc(const dsq_desc *d, const void *packed_device, size_t bytes, const void *x, void *y,
+                             int batch, void *stream);
 
 /* Static, never-NULL text for a status code. */
 DSQ_API const char *dsq_status_string(int status);
