@@ -4,29 +4,28 @@
 // One CTA per row tile (contiguous rows of about equal cost, one tile per
 // SM, from a host schedule built at create).  Warp (rg, cw) owns slot
 // s = 32*cw + lane of rows r0 + rg, r0 + rg + R, ...: each lane streams that
-// slot's 16-byte record (and, for affine rows, the zero byte) straight from
-// HBM with 16-byte loads, U rows per batch of loads and two batches in flight
-// (register double buffering), decodes 32 weights against x held in
-// registers, and the warp reduces the row's partial into shared memory.
-// Meanwhile one thread has started a background bulk copy of x, the tile's
-// CSR entries and its outlier-piece lists into shared memory; after the dense
-// loop the warps reduce the pieces (runs of <= 256 CSR entries of one row)
-// from there, and one thread per row adds the column partials and the row's
-// piece sums, in a fixed order, and stores y.
+// slot's 16-byte record (and the word holding its zero byte or centroid)
+// straight from HBM -- the first rows before the kernel waits on the
+// previous one in the stream, since the packed weights never depend on it --
+// decodes 32 weights against its 32 columns of x held in registers, and the
+// warp reduces the row's partial into shared memory.  Meanwhile one thread
+// has started a background bulk copy of x, the tile's CSR entries and its
+// outlier-piece lists into shared memory; after the dense loop every thread
+// sums whole pieces (runs of <= 31 CSR entries of one row) from there, and
+// one thread per row adds the column partials and the row's piece sums, in a
+// fixed order, and stores y.
 //
-// (A shared-memory ring fed by bulk copies was measured slower here than
-// direct loads: with one CTA per SM streaming its own contiguous range, the
-// loads of 24 warps keep more bytes in flight.)
-//
-// Affine decode.  A 3-bit field at bit p (p + 2 <= 22) of a 32-bit word,
-// masked with AND and read as an fp32, is a subnormal equal to q * 2^(p-149)
-// exactly.  Each lane keeps x[c] * 2^(111-p_c) in registers, so one AND and
-// one FFMA add q * x * 2^-38 exactly (FFMA takes subnormal operands at full
-// rate; nothing here flushes them).  Per group g of 16 columns:
+// Affine decode.  A pair of 3-bit codes sits at the same bit (0, 3 or 6) of
+// both 16-bit halves of a word, or of the word shifted right by 10, so one
+// AND yields two fp16 subnormals q * 2^(k-24), exact.  A mixed-precision FMA
+// (fp32 += fp16 * fp16: the product of two fp16 is exact in fp32) adds
+// q * x * 2^(k-24) into one of three fp32 sums per group, by k; per group g
+// of 16 columns
 //     t_g = sum_c q_c x_c - zero_g * X_g        (X_g = sum of the group's x)
 //     acc += scale_g * t_g
-// i.e. scale*(q - zero) factored out of the group sum; 2^-38 is removed once
-// per row.
+// i.e. scale*(q - zero) factored out of the group sum; 2^-24 is removed once
+// per row.  x stays in its fp16 form in registers: nothing is rounded but
+// the fp32 sums.
 //
 // Table decode.  Every lane of a 2^b-lane segment holds one centroid of the
 // current row (fp32); shfl.idx over that segment reads only the low b bits of
@@ -41,9 +40,14 @@ namespace dsq {
 
 namespace {
 
-constexpr int kMaxWarps = 24;  // worker warps per CTA
+constexpr int kMaxWarps = 24;  // warps per CTA
 constexpr int kThreads = kMaxWarps * 32;
-constexpr int kDepth = 4;      // rows each lane has in flight (cp.async ring stages), a power of 2
+constexpr int kDepth = 4;      // table kernel: rows each lane has in flight (cp.async ring stages), a power of 2
+constexpr int kD = 6;          // affine kernel: rows each lane has in flight (cp.async ring stages)
+constexpr int kHeavyPieces = 32;  // rows with more pieces are summed by a whole warp
+constexpr int kPre = 4;          // affine kernel: ring stages requested before the dependency wait
+// shared-memory header: the mbarrier of the staged CSR + piece lists
+constexpr int kBarCsr = 0;
 constexpr int kStageB = 640;   // ring stage of one warp: 32 x 16-byte slot records + 32 x 4-byte words
 constexpr unsigned kFull = 0xffffffffu;
 constexpr size_t kSmemBudget = 225 * 1024;
@@ -60,58 +64,74 @@ struct B1Params {
     int off_x, off_csr, off_rp, off_pk, off_part, off_psum, off_ring;
 };
 
-// ---- 3-bit field placement (see layout.h) for column c < 30
-__host__ __device__ constexpr int raw_pos3(int c) { return ((c % 10) & 1 ? 16 : 0) + 3 * ((c % 10) >> 1); }
-// masked in the word itself (true) or in the word >> 9 (false)
-__host__ __device__ constexpr bool direct3(int c) { return raw_pos3(c) <= 20; }
-__host__ __device__ constexpr int pos3(int c) { return direct3(c) ? raw_pos3(c) : raw_pos3(c) - 9; }
-
-__device__ __forceinline__ float fld(uint32_t w, uint32_t mask) { return __uint_as_float(w & mask); }
+// ---- 3-bit field placement (layout.h) for column c < 30: bit of the word
+__host__ __device__ constexpr int raw_pos3(int c) {
+    return ((c % 10) & 1 ? 16 : 0) + ((c % 10) >> 1 < 3 ? 3 * ((c % 10) >> 1) : 3 * ((c % 10) >> 1) + 1);
+}
 
 // ---------------------------------------------------------------- aux copy
 
-// x, the tile's CSR entries and its piece / row->piece slices, as 16-byte
-// aligned spans, completing on `aux`.
-__device__ void issue_aux(const B1Params &p, const TileDesc &td, unsigned char *smem, uint64_t *aux,
-                          const __half *x) {
+// The tile's CSR entries and piece / row->piece slices, as 16-byte aligned
+// spans, completing on the CSR barrier.  They belong to the handle (never
+// written by other kernels), so this runs before the dependency wait.
+__device__ void issue_csr(const B1Params &p, const TileDesc &td, unsigned char *smem) {
     const MatrixView &m = p.m;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kBarCsr);
     const int ka = td.k0 & ~3, kb = (td.k1 + 3) & ~3;
     const int ra = td.r0 & ~3, rb = (td.r1 + 1 + 3) & ~3;
     const int pa = td.p0 & ~3, pb = (td.p1 + 1 + 3) & ~3;
-    const uint32_t bytes =
-        (uint32_t)m.cols * 2 + (uint32_t)(kb - ka) * 4 + (uint32_t)(rb - ra) * 4 + (uint32_t)(pb - pa) * 4;
-    mbar_arrive_expect_tx(aux, bytes);
-    bulk_g2s(smem + p.off_x, x, (uint32_t)m.cols * 2, aux);
-    if (kb > ka) bulk_g2s(smem + p.off_csr, m.csr + ka, (uint32_t)(kb - ka) * 4, aux);
-    bulk_g2s(smem + p.off_rp, p.row_piece + ra, (uint32_t)(rb - ra) * 4, aux);
-    bulk_g2s(smem + p.off_pk, p.piece_k + pa, (uint32_t)(pb - pa) * 4, aux);
+    mbar_arrive_expect_tx(bar, (uint32_t)(kb - ka) * 4 + (uint32_t)(rb - ra) * 4 + (uint32_t)(pb - pa) * 4);
+    if (kb > ka) bulk_g2s(smem + p.off_csr, m.csr + ka, (uint32_t)(kb - ka) * 4, bar);
+    bulk_g2s(smem + p.off_rp, p.row_piece + ra, (uint32_t)(rb - ra) * 4, bar);
+    bulk_g2s(smem + p.off_pk, p.piece_k + pa, (uint32_t)(pb - pa) * 4, bar);
 }
 
 // ---------------------------------------------------------------- outliers
 
-// Warp `w` of `nw`: reduce pieces w, w + nw, ... of the tile.
-__device__ __forceinline__ void reduce_pieces(const TileDesc &td, unsigned char *smem, const B1Params &p, int w,
-                                              int nw, int lane) {
-    const __half *xs = reinterpret_cast<const __half *>(smem + p.off_x);
+// f32 += f16 * f16 (the product is exact in fp32).
+__device__ __forceinline__ float mfma(uint16_t a, uint16_t b, float c) {
+    float d;
+    asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float warp_sum(float r) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(kFull, r, o);
+    return r;
+}
+
+// Thread t sums pieces t, t + blockDim, ... of the tile (each <= kPieceMax
+// entries of one row) from the staged CSR entries and x.
+__device__ __forceinline__ void reduce_pieces(const TileDesc &td, unsigned char *smem, const B1Params &p) {
+    const uint16_t *xs = reinterpret_cast<const uint16_t *>(smem + p.off_x);
     const uint32_t *csr = reinterpret_cast<const uint32_t *>(smem + p.off_csr);
     const int32_t *pk = reinterpret_cast<const int32_t *>(smem + p.off_pk);
     float *psum = reinterpret_cast<float *>(smem + p.off_psum);
     const int ka = td.k0 & ~3, pa = td.p0 & ~3;
-    for (int q = td.p0 + w; q < td.p1; q += nw) {
-        const int kb = pk[q - pa], ke = pk[q + 1 - pa];
-        float acc = 0.f;
-        for (int k = kb + lane; k < ke; k += 32) {
-            const uint32_t e = csr[k - ka];
-            acc = fmaf(__half2float(__ushort_as_half((unsigned short)(e >> 16))),
-                       __half2float(xs[e & 0xffffu]), acc);
+    for (int q = td.p0 + threadIdx.x; q < td.p1; q += blockDim.x) {
+        const int kb = pk[q - pa] - ka, ke = pk[q + 1 - pa] - ka;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        int k = kb;
+        for (; k + 3 < ke; k += 4) {
+            const uint32_t e0 = csr[k], e1 = csr[k + 1], e2 = csr[k + 2], e3 = csr[k + 3];
+            a0 = mfma((uint16_t)(e0 >> 16), xs[e0 & 0xffffu], a0);
+            a1 = mfma((uint16_t)(e1 >> 16), xs[e1 & 0xffffu], a1);
+            a2 = mfma((uint16_t)(e2 >> 16), xs[e2 & 0xffffu], a2);
+            a3 = mfma((uint16_t)(e3 >> 16), xs[e3 & 0xffffu], a3);
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-        if (lane == 0) psum[q - td.p0] = acc;
+        for (; k < ke; k++) {
+            const uint32_t e0 = csr[k];
+            a0 = mfma((uint16_t)(e0 >> 16), xs[e0 & 0xffffu], a0);
+        }
+        psum[q - td.p0] = (a0 + a1) + (a2 + a3);
     }
 }
 
-// y[r] = fp16(dense_scale * sum_c part[i][c] + sum of the row's piece sums).
+// y[r] = fp16(dense_scale * sum_c part[i][c] + sum of the row's piece sums),
+// in a fixed order per row.  Warp w takes rows 32w + lane, 32w + lane + 32W,
+// ...: a lane sums the pieces of a row with <= kHeavyPieces of them, the
+// whole warp those of a longer row.
 __device__ __forceinline__ void finalize(const TileDesc &td, const unsigned char *smem, const B1Params &p,
                                          float dense_scale, __half *y) {
     const float *part = reinterpret_cast<const float *>(smem + p.off_part);
@@ -119,47 +139,83 @@ __device__ __forceinline__ void finalize(const TileDesc &td, const unsigned char
     const int32_t *rp = reinterpret_cast<const int32_t *>(smem + p.off_rp);
     const int ra = td.r0 & ~3;
     const int nrows = td.r1 - td.r0;
-    for (int i = threadIdx.x; i < nrows; i += blockDim.x) {
-        float acc = 0.f;
-        for (int c = 0; c < p.C; c++) acc += part[(size_t)i * p.C + c];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int i0 = 32 * warp; i0 < nrows; i0 += 32 * nw) {
+        const int i = i0 + lane;
+        int q0 = 0, q1 = 0;
+        if (i < nrows) {
+            q0 = rp[td.r0 + i - ra];
+            q1 = rp[td.r0 + i + 1 - ra];
+        }
+        const bool heavy = q1 - q0 > kHeavyPieces;
         float o = 0.f;
-        const int q0 = rp[td.r0 + i - ra], q1 = rp[td.r0 + i + 1 - ra];
-        for (int q = q0; q < q1; q++) o += psum[q - td.p0];
-        y[td.r0 + i] = __float2half_rn(fmaf(acc, dense_scale, o));
+        if (!heavy)
+            for (int q = q0; q < q1; q++) o += psum[q - td.p0];
+        unsigned hm = __ballot_sync(kFull, heavy);
+        while (hm) {
+            const int src = __ffs(hm) - 1;
+            hm &= hm - 1;
+            const int h0 = __shfl_sync(kFull, q0, src), h1 = __shfl_sync(kFull, q1, src);
+            float t = 0.f;
+            for (int q = h0 + lane; q < h1; q += 32) t += psum[q - td.p0];
+            t = warp_sum(t);
+            if (lane == src) o = t;
+        }
+        if (i < nrows) {
+            float acc = 0.f;
+            for (int c = 0; c < p.C; c++) acc += part[(size_t)i * p.C + c];
+            y[td.r0 + i] = __float2half_rn(fmaf(acc, dense_scale, o));
+        }
     }
 }
 
 // ---------------------------------------------------------------- row decoders
 
-// Affine 3-bit slot record v (3 code words + scale pair) and zero byte zb:
-// scale_A*(sum_A q x - zA X_A) + scale_B*(...), in units of 2^-38.
-__device__ __forceinline__ float decode_aff3(const uint4 v, uint32_t zb, const float (&xr)[32], float XAt,
+// lo += the low halves' product, hi += the high halves' (fp16 pairs p, x).
+__device__ __forceinline__ void mfma_pair(float &lo, float &hi, uint32_t p, uint32_t xh) {
+    asm("{\n\t.reg .f16 pl, ph, xl, xh;\n\t"
+        "mov.b32 {pl, ph}, %2;\n\tmov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, pl, xl, %0;\n\tfma.rn.f32.f16 %1, ph, xh, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(p), "r"(xh));
+}
+
+// fp32 value of a small unsigned integer n < 2^23 (exact).
+__device__ __forceinline__ float small_u2f(uint32_t n) { return __uint_as_float(n | 0x4B000000u) - 8388608.f; }
+
+// Affine 3-bit slot record v (3 code words + scale pair), zero byte zb, the
+// lane's 32 columns of x as fp16 pairs xh[m] = (x[2m], x[2m+1]) and the
+// group sums of x times 2^-24: returns
+// scale_A*(sum_A q x - zA X_A) + scale_B*(...), in units of 2^-24.
+__device__ __forceinline__ float decode_aff3(const uint4 v, uint32_t zb, const uint32_t (&xh)[16], float XAt,
                                              float XBt) {
-    const uint32_t a[3] = {v.x, v.y, v.z};
-    const uint32_t b[3] = {a[0] >> 9, a[1] >> 9, a[2] >> 9};
-    float pa0 = 0.f, pa1 = 0.f, pb0 = 0.f, pb1 = 0.f;
+    const uint32_t w[3] = {v.x, v.y, v.z};
+    const uint32_t sh[3] = {v.x >> 10, v.y >> 10, v.z >> 10};
+    float acc[2][3][2];  // [group][k / 3][low, high half]
 #pragma unroll
-    for (int c = 0; c < 30; c++) {
-        const uint32_t w = direct3(c) ? a[c / 10] : b[c / 10];
-        const float f = fld(w, 7u << pos3(c));
-        if (c < 16) {
-            if (c & 1) pa1 = fmaf(f, xr[c], pa1); else pa0 = fmaf(f, xr[c], pa0);
-        } else {
-            if (c & 1) pb1 = fmaf(f, xr[c], pb1); else pb0 = fmaf(f, xr[c], pb0);
-        }
+    for (int g = 0; g < 2; g++)
+#pragma unroll
+        for (int k = 0; k < 3; k++) acc[g][k][0] = acc[g][k][1] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 15; m++) {  // pair m = columns 2m, 2m+1: word m/5, slot j = m%5
+        const int i = m / 5, j = m % 5, k = j < 3 ? j : j - 3;
+        const uint32_t pr = (j < 3 ? w[i] : sh[i]) & (0x00070007u << (3 * k));
+        const int g = m < 8 ? 0 : 1;
+        mfma_pair(acc[g][k][0], acc[g][k][1], pr, xh[m]);
     }
-    // columns 30, 31 (group B): bit k at bit 15 / bit 31 of word k
-    pb0 = fmaf(fld(a[0], 1u << 15), xr[30], pb0);
-    pb1 = fmaf(fld(a[1], 1u << 15), xr[30] * 2.f, pb1);
-    pb0 = fmaf(fld(a[2], 1u << 15), xr[30] * 4.f, pb0);
-    pb1 = fmaf(fld(b[0], 1u << 22), xr[31], pb1);
-    pb0 = fmaf(fld(b[1], 1u << 22), xr[31] * 2.f, pb0);
-    pb1 = fmaf(fld(b[2], 1u << 22), xr[31] * 4.f, pb1);
+    // columns 30 (low half) and 31 (high half): bit k is bit 9 / 25 of word k
+    const uint32_t t15 = ((w[0] >> 9) & 0x00010001u) | ((w[1] >> 8) & 0x00020002u) | ((w[2] >> 7) & 0x00040004u);
+    mfma_pair(acc[1][0][0], acc[1][0][1], t15, xh[15]);
+    float t[2];
+#pragma unroll
+    for (int g = 0; g < 2; g++)
+        t[g] = fmaf(acc[g][2][0] + acc[g][2][1], 0x1p-6f,
+                    fmaf(acc[g][1][0] + acc[g][1][1], 0x1p-3f, acc[g][0][0] + acc[g][0][1]));
     const float sA = __half2float(__ushort_as_half((unsigned short)(v.w & 0xffffu)));
     const float sB = __half2float(__ushort_as_half((unsigned short)(v.w >> 16)));
-    const float zA = (float)(zb & 15u), zB = (float)(zb >> 4);
-    const float r = sA * fmaf(-zA, XAt, pa0 + pa1);
-    return fmaf(sB, fmaf(-zB, XBt, pb0 + pb1), r);
+    const float zA = small_u2f(zb & 15u), zB = small_u2f((zb >> 4) & 15u);
+    const float r = sA * fmaf(-zA, XAt, t[0]);
+    return fmaf(sB, fmaf(-zB, XBt, t[1]), r);
 }
 
 // Table slot: code words w[0..BITS-1], this row's centroid held by the lane.
@@ -180,55 +236,196 @@ __device__ __forceinline__ float decode_lut(const uint32_t (&w)[4], float tv, co
             const int sh = raw_pos3(c);
             acc[c & 3] = fmaf(__shfl_sync(kFull, tv, sh ? (int)(wd >> sh) : (int)wd, 8), xr[c], acc[c & 3]);
         }
-        const int q30 = (int)(((w[0] >> 15) & 1u) | ((w[1] >> 14) & 2u) | ((w[2] >> 13) & 4u));
-        const int q31 = (int)((w[0] >> 31) | ((w[1] >> 30) & 2u) | ((w[2] >> 29) & 4u));
+        const int q30 = (int)(((w[0] >> 9) & 1u) | ((w[1] >> 8) & 2u) | ((w[2] >> 7) & 4u));
+        const int q31 = (int)(((w[0] >> 25) & 1u) | ((w[1] >> 24) & 2u) | ((w[2] >> 23) & 4u));
         acc[2] = fmaf(__shfl_sync(kFull, tv, q30, 8), xr[30], acc[2]);
         acc[3] = fmaf(__shfl_sync(kFull, tv, q31, 8), xr[31], acc[3]);
     }
     return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
-__device__ __forceinline__ float warp_sum(float r) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(kFull, r, o);
-    return r;
+// ---------------------------------------------------------------- kernels
+
+// Before the dependency wait: one thread sets up the CSR barrier and starts
+// the CSR staging copy.
+__device__ __forceinline__ void begin(const B1Params &p, const TileDesc &td, unsigned char *smem) {
+    if (threadIdx.x == 0) {
+        mbar_init(reinterpret_cast<uint64_t *>(smem + kBarCsr), 1);
+        fence_mbar_init();
+        issue_csr(p, td, smem);
+    }
 }
 
-// ---------------------------------------------------------------- kernel
+// The warps of row group 0 cover every slot: they stage x (with its zero
+// tail) in shared memory for the outlier pass.
+__device__ __forceinline__ void stage_x(unsigned char *smem, const B1Params &p, int s, const uint32_t (&xh)[16]) {
+    if (s < p.m.slots) {
+        uint4 *dst = reinterpret_cast<uint4 *>(smem + p.off_x + 64 * s);
+#pragma unroll
+        for (int k = 0; k < 4; k++) dst[k] = make_uint4(xh[4 * k], xh[4 * k + 1], xh[4 * k + 2], xh[4 * k + 3]);
+    }
+}
 
-template <int KIND>  // 0: affine 3-bit, 3: LUT 3-bit, 4: LUT 4-bit
+// Wait (warp-wide, bounded) for a staged copy; a timeout is reported.
+__device__ __forceinline__ bool wait_stage(unsigned char *smem, int bar, const B1Params &p) {
+    if (mbar_wait_warp(reinterpret_cast<uint64_t *>(smem + bar), 0)) return true;
+    if ((threadIdx.x & 31) == 0) report(p.status, kStatusTimeout);
+    return false;
+}
+
+// This lane's 32 columns of x (slot s) as 16 fp16 pairs, straight from
+// global memory through the read-only path (x is not written while the
+// kernel runs; the row-group warps of an SM share its lines in L1); columns
+// past N read 0.
+__device__ __forceinline__ void x_pairs(const __half *x, int s, int cols, uint32_t (&xh)[16]) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (s * 32 + 8 * k < cols) q = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)s * 32) + k);
+        xh[4 * k] = q.x;
+        xh[4 * k + 1] = q.y;
+        xh[4 * k + 2] = q.z;
+        xh[4 * k + 3] = q.w;
+    }
+}
+
+// Predicated per-lane asynchronous copies.
+__device__ __forceinline__ void cp_async16_if(uint32_t dst, const void *src, bool p) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t"
+        "@p cp.async.cg.shared.global [%0], [%1], 16;\n\t}" ::"r"(dst),
+        "l"(src), "r"((int)p)
+        : "memory");
+}
+__device__ __forceinline__ void cp_async4_if(uint32_t dst, const void *src, bool p) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t"
+        "@p cp.async.ca.shared.global [%0], [%1], 4;\n\t}" ::"r"(dst),
+        "l"(src), "r"((int)p)
+        : "memory");
+}
+
+// Affine 3-bit rows.  Each lane copies its slot's 16-byte record and the
+// word holding its zero byte for the rows kD ahead into this warp's ring
+// (cp.async, one commit group per row) and reads back exactly what it copied.
 __global__ void __launch_bounds__(kThreads, 1)
-b1_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
-    constexpr bool LUT = KIND != 0;
-    constexpr int BITS = KIND == 4 ? 4 : 3;
-    constexpr int K = 1 << BITS;
-    constexpr int NW = LUT ? BITS : 4;  // 32-bit words loaded per slot and row
+b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
     extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t *aux = reinterpret_cast<uint64_t *>(smem);
     const MatrixView &m = p.m;
     const int S = m.slots, C = p.C, R = p.R;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5;
+    const TileDesc td = p.tiles[blockIdx.x];
+    const int nrows = td.r1 - td.r0;
+    const int cw = warp % C, rg = warp / C;
+    const int s = cw * 32 + lane;
+    // lanes past the last slot re-copy slot S-1 (same sectors); their x is 0
+    const int sc = s < S ? s : S - 1;
+    const int nj = rg < nrows ? (nrows - rg + R - 1) / R : 0;  // rows of this warp
+    const size_t step = (size_t)R * m.row_words * 4;            // bytes between this warp's rows
+    const unsigned char *src = reinterpret_cast<const unsigned char *>(m.dense) +
+                               ((size_t)td.r0 + rg) * m.row_words * 4 + 16 * sc;
+    const int zoff = ((16 * S + sc) & ~3) - 16 * sc;  // zero word, relative to the record
+    const int zsh = 8 * (sc & 3);
+    const uint32_t ring = smem_u32(smem + p.off_ring + (size_t)warp * kD * kStageB);
+    const uint32_t rs = ring + 16 * lane, ra = ring + 512 + 4 * lane;
+    begin(p, td, smem);
+#pragma unroll
+    for (int d = 0; d < kPre; d++) {
+        cp_async16_if(rs + d * kStageB, src, d < nj);
+        cp_async4_if(ra + d * kStageB, src + zoff, d < nj);
+        cp_async_commit();
+        src += step;
+    }
+
+    // x (and y) belong to the surrounding program: wait for the previous
+    // kernel in the stream before touching them.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    {
+        uint32_t xh[16];
+        x_pairs(x, s, m.cols, xh);  // requested ahead of the rest of the ring
+#pragma unroll
+        for (int d = kPre; d < kD; d++) {
+            cp_async16_if(rs + d * kStageB, src, d < nj);
+            cp_async4_if(ra + d * kStageB, src + zoff, d < nj);
+            cp_async_commit();
+            src += step;
+        }
+        float XA = 0.f, XB = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&xh[i]));
+            if (i < 8) XA += f.x + f.y;
+            else XB += f.x + f.y;
+        }
+        const float XAt = XA * 0x1p-24f, XBt = XB * 0x1p-24f;
+        if (rg == 0) stage_x(smem, p, s, xh);
+
+        float *part = reinterpret_cast<float *>(smem + p.off_part) + (size_t)rg * C + cw;
+        const size_t pstep = (size_t)R * C;
+        int j = 0;
+        for (; j + kD <= nj; j += kD) {
+#pragma unroll
+            for (int d = 0; d < kD; d++) {
+                cp_async_wait<kD - 1>();  // row j + d has landed
+                const uint4 v = lds128(rs + d * kStageB);
+                const uint32_t zw = lds32(ra + d * kStageB);
+                const float r = warp_sum(decode_aff3(v, zw >> zsh, xh, XAt, XBt));
+                part[0] = r;  // every lane holds the sum; the stores coincide
+                part += pstep;
+                // refill the stage just read with row j + d + kD
+                const bool more = j + d + kD < nj;
+                cp_async16_if(rs + d * kStageB, src, more);
+                cp_async4_if(ra + d * kStageB, src + zoff, more);
+                cp_async_commit();
+                src += step;
+            }
+        }
+        cp_async_wait<0>();
+        for (int d = 0; j < nj; j++, d++) {
+            const uint4 v = lds128(rs + d * kStageB);
+            const uint32_t zw = lds32(ra + d * kStageB);
+            const float r = warp_sum(decode_aff3(v, zw >> zsh, xh, XAt, XBt));
+            part[0] = r;
+            part += pstep;
+        }
+    }
+    __syncthreads();  // x staged
+    // the outliers, from the staged CSR entries
+    if (wait_stage(smem, kBarCsr, p)) reduce_pieces(td, smem, p);
+    __syncthreads();
+    finalize(td, smem, p, 0x1p24f, y);
+}
+
+template <int KIND>  // 3: LUT 3-bit, 4: LUT 4-bit
+__global__ void __launch_bounds__(kThreads, 1)
+b1_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
+    constexpr int BITS = KIND == 4 ? 4 : 3;
+    constexpr int K = 1 << BITS;
+    constexpr int NW = BITS;  // 32-bit code words per slot and row
+    extern __shared__ __align__(128) unsigned char smem[];
+    const MatrixView &m = p.m;
+    const int S = m.slots, C = p.C, R = p.R;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const TileDesc td = p.tiles[blockIdx.x];
     const int nrows = td.r1 - td.r0;
     const int cw = warp % C, rg = warp / C;
     const int s = cw * 32 + lane;
     const bool valid = s < S;
 
-    // Per-lane asynchronous copy pipeline: each lane copies its own slot
-    // record (and the word holding its zero byte, or its row's centroid) for
-    // the rows kDepth ahead into this warp's ring, and later reads back
-    // exactly what it copied -- no barrier, only cp.async.wait_group.  The
-    // weights do not depend on the previous kernel in the stream, so the
-    // first copies go out before the dependency wait.
+    // Per-lane asynchronous copy pipeline: each lane copies its own slot's
+    // code words (and the word holding its row's centroid) for the rows
+    // kDepth ahead into this warp's ring, and later reads back exactly what
+    // it copied -- no barrier, only cp.async.wait_group.
     const uint32_t ring = smem_u32(smem + p.off_ring + (size_t)warp * kDepth * kStageB);
     const uint32_t ring_s = ring + 16 * lane, ring_a = ring + 512 + 4 * lane;
-    const size_t row_step = (size_t)R * m.row_words * 4;  // bytes between this warp's rows
+    const size_t row_step = (size_t)R * m.row_words * 4;
     const unsigned char *rec = reinterpret_cast<const unsigned char *>(m.dense) +
-                               ((size_t)td.r0 + rg) * m.row_words * 4;  // next row to copy
+                               ((size_t)td.r0 + rg) * m.row_words * 4;
     const unsigned char *tabp = reinterpret_cast<const unsigned char *>(m.table) +
                                 ((size_t)(td.r0 + rg) * K + (lane & (K - 1))) * 2 - 2 * (lane & 1);
-    const int nj = rg < nrows ? (nrows - rg + R - 1) / R : 0;  // rows of this warp
+    const int nj = rg < nrows ? (nrows - rg + R - 1) / R : 0;
     int issued = 0;
     auto issue = [&](int d) {
         if (issued < nj) {
@@ -240,76 +437,41 @@ b1_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
 #pragma unroll
                     for (int k = 0; k < NW; k++) cp_async4(st + 4 * k, rec + 4 * ((size_t)k * S + s));
                 }
-                if (!LUT) cp_async4(sa, rec + ((16 * S + s) & ~3));  // word holding the zero byte
             }
             // the 4-byte word holding this lane's centroid (table rows are 16/32-byte aligned)
-            if (LUT) cp_async4(sa, tabp);
+            cp_async4(sa, tabp);
             rec += row_step;
             tabp += (size_t)R * K * 2;
         }
         issued++;
         cp_async_commit();
     };
+    begin(p, td, smem);
 #pragma unroll
     for (int d = 0; d < kDepth; d++) issue(d);
 
-    // x (and y) belong to the surrounding program: wait for the previous
-    // kernel in the stream before touching them.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (threadIdx.x == 0) {
-        mbar_init(aux, 1);
-        fence_mbar_init();
-    }
-    // zero the padding columns of x in shared memory (the bulk copy fills < N)
-    for (int i = m.cols / 8 + threadIdx.x; i < S * 4; i += blockDim.x)
-        reinterpret_cast<uint4 *>(smem + p.off_x)[i] = make_uint4(0u, 0u, 0u, 0u);
-    __syncthreads();
-    if (threadIdx.x == 0) issue_aux(p, td, smem, aux, x);
-    float *part = reinterpret_cast<float *>(smem + p.off_part);
 
-    // this lane's 32 columns of x from global memory (chunks past N read 0)
-    float xr[32];
+    {
+        float xr[32];
+        {
+            uint32_t xh[16];
+            x_pairs(x, s, m.cols, xh);
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
-        uint4 q = make_uint4(0u, 0u, 0u, 0u);
-        if (valid && s * 32 + 8 * k < m.cols) q = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)s * 32) + k);
-        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int t = 0; t < 4; t++) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&qw[t]));
-            xr[8 * k + 2 * t] = f.x;
-            xr[8 * k + 2 * t + 1] = f.y;
-        }
-    }
-    float XAt = 0.f, XBt = 0.f;
-    if (!LUT) {
-        float XA = 0.f, XB = 0.f;
-#pragma unroll
-        for (int c = 0; c < 32; c++) {
-            if (c < 16) XA += xr[c]; else XB += xr[c];
-            const int pc = c < 30 ? pos3(c) : (c == 30 ? 15 : 22);
-            xr[c] *= __uint_as_float((uint32_t)(127 + 111 - pc) << 23);
-        }
-        XAt = XA * 0x1p-38f;
-        XBt = XB * 0x1p-38f;
-    }
-
-    int i = rg;
-    for (int j = 0; j < nj; j++, i += R) {
-        const int d = j & (kDepth - 1);
-        cp_async_wait<kDepth - 1>();  // this lane's copies for row j have landed
-        const uint32_t st = ring_s + d * kStageB, sa = ring_a + d * kStageB;
-        float r = 0.f;
-        if (!LUT) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            uint32_t zb = 0u;
-            if (valid) {
-                v = lds128(st);
-                zb = (lds32(sa) >> (8 * (s & 3))) & 0xffu;
+            for (int i = 0; i < 16; i++) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&xh[i]));
+                xr[2 * i] = f.x;
+                xr[2 * i + 1] = f.y;
             }
-            r = decode_aff3(v, zb, xr, XAt, XBt);
-        } else {
+            if (rg == 0) stage_x(smem, p, s, xh);
+        }
+        float *part = reinterpret_cast<float *>(smem + p.off_part);
+        int i = rg;
+        for (int j = 0; j < nj; j++, i += R) {
+            const int d = j & (kDepth - 1);
+            cp_async_wait<kDepth - 1>();  // this lane's copies for row j have landed
+            const uint32_t st = ring_s + d * kStageB, sa = ring_a + d * kStageB;
             uint32_t w4[4] = {0u, 0u, 0u, 0u};
             if (valid) {
                 if (NW == 4) {
@@ -321,18 +483,17 @@ b1_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
                 }
             }
             const float tv = __half2float(__ushort_as_half((unsigned short)(lds32(sa) >> (16 * (lane & 1)))));
-            r = decode_lut<BITS>(w4, tv, xr);
+            float r = decode_lut<BITS>(w4, tv, xr);
+            r = warp_sum(r);
+            if (lane == 0) part[(size_t)i * C + cw] = r;
+            issue(d);  // refill this stage (its data has been consumed)
         }
-        r = warp_sum(r);
-        if (lane == 0) part[(size_t)i * C + cw] = r;
-        issue(d);  // refill this stage (its data has been consumed)
+        cp_async_wait<0>();
     }
-    cp_async_wait<0>();
-
-    if (mbar_wait_warp(aux, 0)) reduce_pieces(td, smem, p, warp, nwarps, lane);
-    else if (lane == 0) report(p.status, kStatusTimeout);
+    __syncthreads();  // x staged
+    if (wait_stage(smem, kBarCsr, p)) reduce_pieces(td, smem, p);
     __syncthreads();
-    finalize(td, smem, p, LUT ? 1.0f : 0x1p38f, y);
+    finalize(td, smem, p, 1.0f, y);
 }
 
 enum Kind { kNone = -1, kAff3 = 0, kLut3 = 3, kLut4 = 4 };
@@ -371,9 +532,10 @@ bool plan_b1(const dsq_handle_s *h, B1Params *out, size_t *smem_bytes) {
     p.off_part = (int)off;
     off = align_sz(off + (size_t)sc.max_rows * p.C * 4, 16);
     p.off_psum = (int)off;
-    off = align_sz(off + (size_t)(sc.max_pieces + 1) * 4, 128);
+    off = align_sz(off + (size_t)(sc.max_pieces + 1) * 4, 16);
+    off = align_sz(off, 128);
     p.off_ring = (int)off;
-    off += (size_t)p.C * p.R * kDepth * kStageB;
+    off += (size_t)p.C * p.R * (b1_kind(m, 1) == kAff3 ? kD : kDepth) * kStageB;
     if (off > kSmemBudget) return false;
     *out = p;
     *smem_bytes = off;
@@ -421,12 +583,14 @@ int build_schedule(dsq_handle_s *h, const int32_t *rp) {
 
     const int tiles_target = std::max(1, std::min(h->sm_count, m.rows));
     double total = 0;
-    for (int i = 0; i < m.rows; i++) total += 4.0 * m.row_words + 8.0 * (rp[i + 1] - rp[i]) + 64.0;
+    // Cost of a row: its record bytes plus a charge per outlier.
+    auto row_cost = [&](int i) { return 4.0 * m.row_words + 4.0 * (rp[i + 1] - rp[i]) + 64.0; };
+    for (int i = 0; i < m.rows; i++) total += row_cost(i);
     std::vector<TileDesc> tiles;
     int r0 = 0;
     double acc = 0, done = 0;
     for (int i = 0; i < m.rows; i++) {
-        const double c = 4.0 * m.row_words + 8.0 * (rp[i + 1] - rp[i]) + 64.0;
+        const double c = row_cost(i);
         const bool over_csr = i > r0 && rp[i + 1] - rp[r0] > kTileCsrCap;
         const bool due = acc > 0 && (done + acc + c / 2) * tiles_target >= total * (tiles.size() + 1);
         if (i > r0 && (over_csr || (due && (int)tiles.size() + 1 < tiles_target))) {
@@ -462,9 +626,9 @@ void free_schedule(dsq_handle_s *h) {
 
 // Per-device kernel attributes; called by dsq_create with the device current.
 int fused_prepare(dsq_handle_s *) {
-    int rc = set_smem_attr(b1_kernel<kAff3>);
-    if (rc == DSQ_OK) rc = set_smem_attr(b1_kernel<kLut3>);
-    if (rc == DSQ_OK) rc = set_smem_attr(b1_kernel<kLut4>);
+    int rc = set_smem_attr(b1_aff3_kernel);
+    if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<kLut3>);
+    if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<kLut4>);
     return rc;
 }
 
@@ -494,9 +658,9 @@ int launch_gemv_fused(const dsq_handle_s *h, const __half *x, __half *y, int bat
     cfg.numAttrs = 1;
     cudaError_t e;
     switch (kind) {
-        case kAff3: e = cudaLaunchKernelEx(&cfg, b1_kernel<kAff3>, p, x, y); break;
-        case kLut3: e = cudaLaunchKernelEx(&cfg, b1_kernel<kLut3>, p, x, y); break;
-        default: e = cudaLaunchKernelEx(&cfg, b1_kernel<kLut4>, p, x, y); break;
+        case kAff3: e = cudaLaunchKernelEx(&cfg, b1_aff3_kernel, p, x, y); break;
+        case kLut3: e = cudaLaunchKernelEx(&cfg, b1_lut_kernel<kLut3>, p, x, y); break;
+        default: e = cudaLaunchKernelEx(&cfg, b1_lut_kernel<kLut4>, p, x, y); break;
     }
     return e == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
 }

@@ -36,8 +36,10 @@ struct TileDesc {
 // Schedule of the batch-1 kernels, built at create for the device's SM
 // count.  Outliers are cut into "pieces": runs of at most kPieceMax entries
 // of one row; piece p covers CSR entries [piece_k[p], piece_k[p+1]) and row
-// r owns pieces [row_piece[r], row_piece[r+1]).
-constexpr int kPieceMax = 256;
+// r owns pieces [row_piece[r], row_piece[r+1]).  One lane sums a piece; an
+// odd kPieceMax keeps the lanes walking consecutive pieces of a long row on
+// distinct shared-memory banks.
+constexpr int kPieceMax = 31;
 struct Schedule {
     int n_tiles = 0;
     int max_rows = 0;     // rows of the largest tile

@@ -26,12 +26,14 @@
 //
 // Code bits inside a slot.  4-bit: column c in word c/8, bits 4(c%8)..+3.
 // 3-bit: word w (0..2) holds columns 10w..10w+9 as five adjacent pairs; pair
-// j (columns 10w+2j, 10w+2j+1) sits at bits 3j (low half) and 16+3j (high
-// half), so one mask pulls both codes of a pair into the two fp16 halves of
-// a word.  Every field also lies in bits 0..22 of the word, or of the word
-// shifted right by 9, so an AND alone turns it into an exact fp32
-// subnormal.  Columns 30 and 31 use the spare bits: bit k of column 30 is
-// bit 15 of word k, bit k of column 31 is bit 31 of word k.
+// j (columns 10w+2j, 10w+2j+1) sits at half-word bit h_j of the low half
+// (even column) and of the high half (odd column), h = 0, 3, 6, 10, 13.  One
+// mask therefore pulls both codes of a pair into the two 16-bit halves of a
+// word, and since pairs 0..2 lie in bits 0..9 of each half -- and pairs 3, 4
+// do in the word shifted right by 10 -- an AND alone turns a pair into two
+// exact fp16 subnormals (q * 2^(h-24)).  Columns 30 and 31 use the spare
+// bits: bit k of column 30 is bit 9 of word k, bit k of column 31 is bit 25
+// of word k.
 #pragma once
 #include <stdint.h>
 
@@ -87,13 +89,13 @@ __host__ __device__ inline void code_bit_place(int bits, int c, int k, int *word
         return;
     }
     if (c < 30) {
-        const int t = c % 10;
+        const int t = c % 10, j = t >> 1;
         *word = c / 10;
-        *pos = (t & 1 ? 16 : 0) + 3 * (t >> 1) + k;
+        *pos = (t & 1 ? 16 : 0) + (j < 3 ? 3 * j : 3 * j + 1) + k;
         return;
     }
     *word = k;
-    *pos = c == 30 ? 15 : 31;
+    *pos = c == 30 ? 9 : 25;
 }
 
 // Word index (inside a record) of code word p of slot s.

@@ -11,7 +11,6 @@
 namespace dsq {
 
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait
-constexpr uint32_t kSuspendHintNs = 100000;  // per try_wait, while the phase is incomplete
 constexpr int kStatusTimeout = 1;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -42,17 +41,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
         : "memory");
 }
 
-// One test of the phase; while it is incomplete the thread may sleep up to
-// the hinted time (it wakes when the phase completes), so waiting warps do
-// not take issue slots from working ones.
+// One test of the phase (mbarrier.try_wait: the hardware may hold the
+// thread briefly while the phase is incomplete; it resumes as soon as the
+// phase completes).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }

@@ -150,7 +150,7 @@ __device__ __forceinline__ void decode_slot_f16(uint4 v, uint32_t zb, uint32_t (
     asm("prmt.b32 %0, %1, %1, 0x1010;" : "=r"(sA) : "r"(v.w));
     asm("prmt.b32 %0, %1, %1, 0x3232;" : "=r"(sB) : "r"(v.w));
     const uint32_t a[3] = {v.x, v.y, v.z};
-    const uint32_t b[3] = {v.x >> 9, v.y >> 9, v.z >> 9};
+    const uint32_t b[3] = {v.x >> 10, v.y >> 10, v.z >> 10};
 #pragma unroll
     for (int P = 0; P < 15; P++) {
         const int w = P / 5, j = P % 5;
@@ -159,7 +159,8 @@ __device__ __forceinline__ void decode_slot_f16(uint4 v, uint32_t zb, uint32_t (
         const __half2 qz = __hfma2(u2h(h), cs[t], P < 8 ? dA[t] : dB[t]);
         o[P] = h2u(__hmul2(qz, u2h(P < 8 ? sA : sB)));
     }
-    const uint32_t t15 = ((a[0] >> 15) & 0x00010001u) | ((a[1] >> 14) & 0x00020002u) | ((a[2] >> 13) & 0x00040004u);
+    // columns 30 (low half) and 31 (high half): bit k at bits 9 / 25 of word k
+    const uint32_t t15 = ((a[0] >> 9) & 0x00010001u) | ((a[1] >> 8) & 0x00020002u) | ((a[2] >> 7) & 0x00040004u);
     o[15] = h2u(__hmul2(__hadd2(u2h(t15 | kMagic), nB), u2h(sB)));
 }
 

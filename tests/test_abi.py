@@ -171,8 +171,8 @@ def unpack_blob(blob: bytes):
             return c // 8, 4 * (c % 8) + k
         if c < 30:
             t = c % 10
-            return c // 10, (16 if t % 2 else 0) + 3 * (t // 2) + k
-        return k, (15 if c == 30 else 31)
+            return c // 10, (16 if t % 2 else 0) + [0, 3, 6, 10, 13][t // 2] + k
+        return k, (9 if c == 30 else 25)
 
     codes = np.zeros((rows, cols), np.uint8)
     for s in range(S):
@@ -228,22 +228,20 @@ def test_layout_round_trip(bits, mode, cols):
 
 def test_three_bit_fields():
     """3-bit placement: columns 2j and 2j+1 of a word's ten sit 16 bits apart
-    (one mask puts both into the two fp16 halves, each at bit <= 12 of its
-    half); every field lies in bits 0..22 of its word or of the word >> 9 (an
-    AND then yields an exact fp32 subnormal); columns 30/31 fill bits 15/31;
-    the 96 bits are used once each."""
+    (one mask puts both into the two 16-bit halves); every pair lies in bits
+    0..9 of its halves, either in the word or in the word >> 10, so an AND
+    alone makes two exact fp16 subnormals; columns 30/31 fill bits 9/25; the
+    96 bits are used once each."""
     place = {}
     for c in range(32):
         for k in range(3):
             if c < 30:
                 t = c % 10
-                place[c, k] = (c // 10, (16 if t % 2 else 0) + 3 * (t // 2) + k)
+                place[c, k] = (c // 10, (16 if t % 2 else 0) + [0, 3, 6, 10, 13][t // 2] + k)
             else:
-                place[c, k] = (k, 15 if c == 30 else 31)
+                place[c, k] = (k, 9 if c == 30 else 25)
     assert len(set(place.values())) == 96
     for c in range(0, 30, 2):
         (w0, p0), (w1, p1) = place[c, 0], place[c + 1, 0]
-        assert w0 == w1 and p1 == p0 + 16 and p0 <= 12
-    for c in range(30):
-        p = place[c, 0][1]
-        assert p + 2 <= 22 or (p - 9 >= 0 and p - 9 + 2 <= 22)
+        assert w0 == w1 and p1 == p0 + 16
+        assert p0 + 2 <= 9 or (p0 >= 10 and p0 - 10 + 2 <= 9)
