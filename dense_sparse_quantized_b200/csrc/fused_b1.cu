@@ -31,6 +31,7 @@
 // current row (fp32); shfl.idx over that segment reads only the low b bits of
 // its index, so a code needs a shift but no mask.
 #include <algorithm>
+#include <type_traits>
 #include <vector>
 
 #include "internal.h"
@@ -46,9 +47,10 @@ constexpr int kDepth = 4;      // table kernel: rows each lane has in flight (cp
 constexpr int kD = 6;          // affine kernel: rows each lane has in flight (cp.async ring stages)
 constexpr int kHeavyPieces = 32;  // rows with more pieces are summed by a whole warp
 constexpr int kPre = 4;          // affine kernel: ring stages requested before the dependency wait
-// shared-memory header: the mbarrier of the staged CSR + piece lists
-constexpr int kBarCsr = 0;
-constexpr int kStageB = 640;   // ring stage of one warp: 32 x 16-byte slot records + 32 x 4-byte words
+// shared-memory header: mbarriers of the staged CSR + piece lists and of the
+// staged x
+constexpr int kBarCsr = 0, kBarX = 8;
+constexpr int kStageB = 640;   // table kernel ring stage of one warp: 32 x 16-byte code words + 32 x 4-byte words
 constexpr unsigned kFull = 0xffffffffu;
 constexpr size_t kSmemBudget = 225 * 1024;
 constexpr int kTileCsrCap = 12288;  // CSR entries per tile (48 KB), unless one row needs more
@@ -246,24 +248,28 @@ __device__ __forceinline__ float decode_lut(const uint32_t (&w)[4], float tv, co
 
 // ---------------------------------------------------------------- kernels
 
-// Before the dependency wait: one thread sets up the CSR barrier and starts
-// the CSR staging copy.
+// Before the dependency wait: one thread sets up the barriers and starts the
+// CSR staging copy.
 __device__ __forceinline__ void begin(const B1Params &p, const TileDesc &td, unsigned char *smem) {
     if (threadIdx.x == 0) {
         mbar_init(reinterpret_cast<uint64_t *>(smem + kBarCsr), 1);
+        mbar_init(reinterpret_cast<uint64_t *>(smem + kBarX), p.C);  // one arrival per column warp
         fence_mbar_init();
         issue_csr(p, td, smem);
     }
+    __syncthreads();
 }
 
 // The warps of row group 0 cover every slot: they stage x (with its zero
-// tail) in shared memory for the outlier pass.
+// tail) in shared memory for the outlier pass and arrive on its barrier.
 __device__ __forceinline__ void stage_x(unsigned char *smem, const B1Params &p, int s, const uint32_t (&xh)[16]) {
     if (s < p.m.slots) {
         uint4 *dst = reinterpret_cast<uint4 *>(smem + p.off_x + 64 * s);
 #pragma unroll
         for (int k = 0; k < 4; k++) dst[k] = make_uint4(xh[4 * k], xh[4 * k + 1], xh[4 * k + 2], xh[4 * k + 3]);
     }
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(reinterpret_cast<uint64_t *>(smem + kBarX));
 }
 
 // Wait (warp-wide, bounded) for a staged copy; a timeout is reported.
@@ -289,25 +295,49 @@ __device__ __forceinline__ void x_pairs(const __half *x, int s, int cols, uint32
     }
 }
 
-// Predicated per-lane asynchronous copies.
-__device__ __forceinline__ void cp_async16_if(uint32_t dst, const void *src, bool p) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t"
-        "@p cp.async.cg.shared.global [%0], [%1], 16;\n\t}" ::"r"(dst),
-        "l"(src), "r"((int)p)
-        : "memory");
+// Calls f(std::integral_constant<int, D>) for D = B .. E-1 (compile-time stage indices).
+template <int B, int E, typename F>
+__device__ __forceinline__ void unroll(F &&f) {
+    if constexpr (B < E) {
+        f(std::integral_constant<int, B>{});
+        unroll<B + 1, E>(f);
+    }
 }
-__device__ __forceinline__ void cp_async4_if(uint32_t dst, const void *src, bool p) {
+
+// Affine 3-bit: ring stage of one warp = the 32 slot records of its group
+// (512 bytes) + the group's 32 zero bytes.
+constexpr int kAffStageB = 544;
+
+// One row of this lane's ring: its slot record (all lanes; source lb + 32)
+// and, on lanes 0 and 1, half of the group's zero bytes (source lb), into
+// stage OFF; predicated on `more`.  One commit group.  (Per-lane copies on
+// the L1 path measured faster here than one bulk copy per warp and row.)
+template <int OFF>
+__device__ __forceinline__ void copy_row(uint32_t rs, uint32_t rz, const unsigned char *lb, int more, int zl) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t"
-        "@p cp.async.ca.shared.global [%0], [%1], 4;\n\t}" ::"r"(dst),
-        "l"(src), "r"((int)p)
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %2, 0;\n\t"
+        "setp.ne.and.b32 q, %3, 0, p;\n\t"
+        "@p cp.async.cg.shared.global [%0+%5], [%1+32], 16;\n\t"
+        "@q cp.async.cg.shared.global [%4+%5], [%1], 16;\n\t"
+        "cp.async.commit_group;\n\t}" ::"r"(rs),
+        "l"(lb), "r"(more), "r"(zl), "r"(rz), "n"(OFF)
         : "memory");
 }
 
-// Affine 3-bit rows.  Each lane copies its slot's 16-byte record and the
-// word holding its zero byte for the rows kD ahead into this warp's ring
-// (cp.async, one commit group per row) and reads back exactly what it copied.
+template <int OFF>
+__device__ __forceinline__ void read_row(uint32_t rs, uint32_t rb, uint4 &v, uint32_t &zb) {
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(rs), "n"(OFF));
+    asm volatile("ld.shared.u8 %0, [%1+%2];" : "=r"(zb) : "r"(rb), "n"(OFF + 512));
+}
+
+// Affine 3-bit rows.  The lanes of warp (rg, cw) stream group cw of rows
+// r0 + rg, r0 + rg + R, ...: each lane copies its slot's 16-byte record and
+// lanes 0, 1 the group's zero bytes, kD rows ahead, into the warp's ring
+// (cp.async, one commit group per row); each lane reads back its record and
+// zero byte.
 __global__ void __launch_bounds__(kThreads, 1)
 b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -318,24 +348,22 @@ b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y)
     const int nrows = td.r1 - td.r0;
     const int cw = warp % C, rg = warp / C;
     const int s = cw * 32 + lane;
-    // lanes past the last slot re-copy slot S-1 (same sectors); their x is 0
-    const int sc = s < S ? s : S - 1;
+    const int nslot = min(32, S - 32 * cw);  // slots in this warp's group
     const int nj = rg < nrows ? (nrows - rg + R - 1) / R : 0;  // rows of this warp
     const size_t step = (size_t)R * m.row_words * 4;            // bytes between this warp's rows
-    const unsigned char *src = reinterpret_cast<const unsigned char *>(m.dense) +
-                               ((size_t)td.r0 + rg) * m.row_words * 4 + 16 * sc;
-    const int zoff = ((16 * S + sc) & ~3) - 16 * sc;  // zero word, relative to the record
-    const int zsh = 8 * (sc & 3);
-    const uint32_t ring = smem_u32(smem + p.off_ring + (size_t)warp * kD * kStageB);
-    const uint32_t rs = ring + 16 * lane, ra = ring + 512 + 4 * lane;
+    // lanes past the group's last slot copy that slot again (same sectors); their x is 0
+    const unsigned char *lb = reinterpret_cast<const unsigned char *>(m.dense) +
+                              ((size_t)td.r0 + rg) * m.row_words * 4 + 4 * kAff3GroupWords * cw +
+                              16 * min(lane, nslot - 1);
+    const int zl = lane < 2;
+    const uint32_t ring = smem_u32(smem + p.off_ring + (size_t)warp * kD * kAffStageB);
+    const uint32_t rs = ring + 16 * lane, rz = ring + 512 + 16 * lane, rb = ring + lane;
     begin(p, td, smem);
-#pragma unroll
-    for (int d = 0; d < kPre; d++) {
-        cp_async16_if(rs + d * kStageB, src, d < nj);
-        cp_async4_if(ra + d * kStageB, src + zoff, d < nj);
-        cp_async_commit();
-        src += step;
-    }
+    unroll<0, kPre>([&](auto dc) {
+        constexpr int d = decltype(dc)::value;
+        copy_row<d * kAffStageB>(rs, rz, lb, d < nj, zl);
+        lb += step;
+    });
 
     // x (and y) belong to the surrounding program: wait for the previous
     // kernel in the stream before touching them.
@@ -345,13 +373,11 @@ b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y)
     {
         uint32_t xh[16];
         x_pairs(x, s, m.cols, xh);  // requested ahead of the rest of the ring
-#pragma unroll
-        for (int d = kPre; d < kD; d++) {
-            cp_async16_if(rs + d * kStageB, src, d < nj);
-            cp_async4_if(ra + d * kStageB, src + zoff, d < nj);
-            cp_async_commit();
-            src += step;
-        }
+        unroll<kPre, kD>([&](auto dc) {
+            constexpr int d = decltype(dc)::value;
+            copy_row<d * kAffStageB>(rs, rz, lb, d < nj, zl);
+            lb += step;
+        });
         float XA = 0.f, XB = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; i++) {
@@ -362,38 +388,37 @@ b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y)
         const float XAt = XA * 0x1p-24f, XBt = XB * 0x1p-24f;
         if (rg == 0) stage_x(smem, p, s, xh);
 
-        float *part = reinterpret_cast<float *>(smem + p.off_part) + (size_t)rg * C + cw;
-        const size_t pstep = (size_t)R * C;
+        uint32_t part = smem_u32(smem + p.off_part) + 4 * (rg * C + cw);
+        const uint32_t pstep = 4 * R * C;
         int j = 0;
         for (; j + kD <= nj; j += kD) {
-#pragma unroll
-            for (int d = 0; d < kD; d++) {
+            unroll<0, kD>([&](auto dc) {
+                constexpr int d = decltype(dc)::value;
                 cp_async_wait<kD - 1>();  // row j + d has landed
-                const uint4 v = lds128(rs + d * kStageB);
-                const uint32_t zw = lds32(ra + d * kStageB);
-                const float r = warp_sum(decode_aff3(v, zw >> zsh, xh, XAt, XBt));
-                part[0] = r;  // every lane holds the sum; the stores coincide
+                uint4 v;
+                uint32_t zb;
+                read_row<d * kAffStageB>(rs, rb, v, zb);
+                const float r = warp_sum(decode_aff3(v, zb, xh, XAt, XBt));
+                // every lane holds the sum; the stores coincide
+                asm volatile("st.shared.f32 [%0], %1;" ::"r"(part), "f"(r) : "memory");
                 part += pstep;
                 // refill the stage just read with row j + d + kD
-                const bool more = j + d + kD < nj;
-                cp_async16_if(rs + d * kStageB, src, more);
-                cp_async4_if(ra + d * kStageB, src + zoff, more);
-                cp_async_commit();
-                src += step;
-            }
+                copy_row<d * kAffStageB>(rs, rz, lb, j + d + kD < nj, zl);
+                lb += step;
+            });
         }
         cp_async_wait<0>();
         for (int d = 0; j < nj; j++, d++) {
-            const uint4 v = lds128(rs + d * kStageB);
-            const uint32_t zw = lds32(ra + d * kStageB);
-            const float r = warp_sum(decode_aff3(v, zw >> zsh, xh, XAt, XBt));
-            part[0] = r;
+            uint4 v;
+            uint32_t zb;
+            read_row<0>(rs + d * kAffStageB, rb + d * kAffStageB, v, zb);
+            const float r = warp_sum(decode_aff3(v, zb, xh, XAt, XBt));
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(part), "f"(r) : "memory");
             part += pstep;
         }
     }
-    __syncthreads();  // x staged
-    // the outliers, from the staged CSR entries
-    if (wait_stage(smem, kBarCsr, p)) reduce_pieces(td, smem, p);
+    // the outliers, from the staged CSR entries and x
+    if (wait_stage(smem, kBarX, p) && wait_stage(smem, kBarCsr, p)) reduce_pieces(td, smem, p);
     __syncthreads();
     finalize(td, smem, p, 0x1p24f, y);
 }
@@ -490,8 +515,7 @@ b1_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) 
         }
         cp_async_wait<0>();
     }
-    __syncthreads();  // x staged
-    if (wait_stage(smem, kBarCsr, p)) reduce_pieces(td, smem, p);
+    if (wait_stage(smem, kBarX, p) && wait_stage(smem, kBarCsr, p)) reduce_pieces(td, smem, p);
     __syncthreads();
     finalize(td, smem, p, 1.0f, y);
 }
@@ -535,7 +559,7 @@ bool plan_b1(const dsq_handle_s *h, B1Params *out, size_t *smem_bytes) {
     off = align_sz(off + (size_t)(sc.max_pieces + 1) * 4, 16);
     off = align_sz(off, 128);
     p.off_ring = (int)off;
-    off += (size_t)p.C * p.R * (b1_kind(m, 1) == kAff3 ? kD : kDepth) * kStageB;
+    off += (size_t)p.C * p.R * (b1_kind(m, 1) == kAff3 ? kD * kAffStageB : kDepth * kStageB);
     if (off > kSmemBudget) return false;
     *out = p;
     *smem_bytes = off;

@@ -27,7 +27,7 @@ __device__ __forceinline__ void load_slot(const MatrixView &m, const uint32_t *r
     for (int p = 0; p < BITS; p++) w[p] = __ldg(rec + code_word_index(BITS, MODE, m.slots, s, p));
     if (MODE == DSQ_MODE_AFFINE_G16) {
         scales = __ldg(rec + scale_word_index(BITS, m.slots, s));
-        zb = __ldg((const uint8_t *)(rec + zero_word_offset(BITS, MODE, m.slots)) + s);
+        zb = __ldg((const uint8_t *)rec + zero_byte_index(BITS, m.slots, s));
     }
 }
 

@@ -15,14 +15,20 @@
 //
 //   LUT_ROW, 3 bit:    3 planes of S words: word p of slot s at [p*S + s]
 //   LUT_ROW, 4 bit:    S uint4 (4 code words) at [4s .. 4s+3]
-//   AFFINE_G16, 3 bit: S uint4 = (code word 0, 1, 2, scale pair) at [4s..]
-//   AFFINE_G16, 4 bit: S uint4 code words, then S scale-pair words at [4S+s]
-//   AFFINE_G16:        then S zero bytes (byte s = zero[2s] | zero[2s+1]<<4)
-//                      starting at word Z = (bits == 3 ? 4S : 5S)
+//   AFFINE_G16, 3 bit: groups of 32 slots, 136 words apart: group g holds
+//                      the zero bytes of its slots (8 words; byte t =
+//                      zero byte of slot 32g + t), then one uint4 per slot
+//                      = (code word 0, 1, 2, scale pair) at [136g + 8 + 4t];
+//                      the last group holds only its S - 32g slots
+//   AFFINE_G16, 4 bit: S uint4 code words, then S scale-pair words at [4S+s],
+//                      then S zero bytes starting at word 5S
 //
-// and the record is padded to a multiple of 4 words, so every record and
-// every uint4 starts on a 16-byte boundary.  A scale pair is
-// scale[2s] | scale[2s+1] << 16 (the two groups of 16 in the slot).
+// A zero byte is zero[2s] | zero[2s+1] << 4, a scale pair is
+// scale[2s] | scale[2s+1] << 16 (the two groups of 16 in the slot).  Records
+// are padded to a multiple of 4 words, so every record and every uint4
+// starts on a 16-byte boundary.  (The 3-bit affine grouping gives the 32
+// lanes that stream one group a single base address: zero bytes at +0,
+// their slot at +32 + 16*lane.)
 //
 // Code bits inside a slot.  4-bit: column c in word c/8, bits 4(c%8)..+3.
 // 3-bit: word w (0..2) holds columns 10w..10w+9 as five adjacent pairs; pair
@@ -66,18 +72,22 @@ static_assert(sizeof(BlobHeader) == kHeaderBytes, "header size");
 
 __host__ __device__ inline int slots_of(int cols) { return (cols + kSlotCols - 1) / kSlotCols; }
 
-// Word offset (inside a record) of the zero bytes; -1 in LUT mode.
-__host__ __device__ inline int zero_word_offset(int bits, int mode, int S) {
-    return mode == 1 ? (bits == 3 ? 4 * S : 5 * S) : -1;
-}
+constexpr int kAff3GroupWords = 136;  // 8 words of zero bytes + 32 slot uint4
 
 __host__ __device__ inline int row_words_of(int bits, int mode, int S) {
     int w;
     if (mode == 0)
         w = bits * S;
+    else if (bits == 3)
+        w = S == 0 ? 0 : kAff3GroupWords * ((S - 1) / 32) + 8 + 4 * (S - 32 * ((S - 1) / 32));
     else
-        w = zero_word_offset(bits, mode, S) + (S + 3) / 4;
+        w = 5 * S + (S + 3) / 4;
     return (w + 3) & ~3;
+}
+
+// Byte offset (inside a record) of the zero byte of slot s (affine only).
+__host__ __device__ inline int zero_byte_index(int bits, int S, int s) {
+    return bits == 3 ? 4 * kAff3GroupWords * (s / 32) + (s % 32) : 4 * 5 * S + s;
 }
 
 // Position of bit k (0 = least significant) of column c's code inside a
@@ -101,12 +111,13 @@ __host__ __device__ inline void code_bit_place(int bits, int c, int k, int *word
 // Word index (inside a record) of code word p of slot s.
 __host__ __device__ inline int code_word_index(int bits, int mode, int S, int s, int p) {
     if (bits == 3 && mode == 0) return p * S + s;
+    if (bits == 3) return kAff3GroupWords * (s / 32) + 8 + 4 * (s % 32) + p;
     return 4 * s + p;
 }
 
 // Word index of the scale pair of slot s (affine only).
 __host__ __device__ inline int scale_word_index(int bits, int S, int s) {
-    return bits == 3 ? 4 * s + 3 : 4 * S + s;
+    return bits == 3 ? code_word_index(3, 1, S, s, 3) : 4 * S + s;
 }
 
 }  // namespace dsq

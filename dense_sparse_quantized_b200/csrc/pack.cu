@@ -166,7 +166,7 @@ extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t 
                     zb |= (uint32_t)half_bits_to_double(zeros[i * G + g]) << (4 * e);
                 }
                 rec[scale_word_index(bits, S, s)] = pair;
-                ((uint8_t *)(rec + zero_word_offset(bits, mode, S)))[s] = (uint8_t)zb;
+                ((uint8_t *)rec)[zero_byte_index(bits, S, s)] = (uint8_t)zb;
             }
         }
     }

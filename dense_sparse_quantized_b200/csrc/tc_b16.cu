@@ -305,8 +305,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, TcParams p, int KS, __half *
                 v[u] = make_uint4(0u, 0u, 0u, 0u);
                 zb[u] = 0u;
                 if (i < nk && slot < p.S && grow < p.rows) {
-                    v[u] = __ldg(reinterpret_cast<const uint4 *>(rec) + slot);
-                    zb[u] = __ldg(reinterpret_cast<const uint8_t *>(rec + 4 * p.S) + slot);
+                    v[u] = __ldg(reinterpret_cast<const uint4 *>(rec + code_word_index(3, 1, p.S, slot, 0)));
+                    zb[u] = __ldg(reinterpret_cast<const uint8_t *>(rec) + zero_byte_index(3, p.S, slot));
                 }
             }
         };

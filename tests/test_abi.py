@@ -174,10 +174,20 @@ def unpack_blob(blob: bytes):
             return c // 10, (16 if t % 2 else 0) + [0, 3, 6, 10, 13][t // 2] + k
         return k, (9 if c == 30 else 25)
 
+    def word_of(s, p_):
+        # word index inside a record of code word p_ (3 = scale pair) of slot s
+        if bits == 3 and mode == 0:
+            return p_ * S + s
+        if bits == 3:
+            return 136 * (s // 32) + 8 + 4 * (s % 32) + p_
+        return 4 * s + p_ if p_ < 4 else 4 * S + s
+
+    def zero_byte(s):
+        return 4 * 136 * (s // 32) + s % 32 if bits == 3 else 4 * 5 * S + s
+
     codes = np.zeros((rows, cols), np.uint8)
     for s in range(S):
-        words = [rec[:, (p_ * S + s) if (bits == 3 and mode == 0) else (4 * s + p_)]
-                 for p_ in range(bits)]
+        words = [rec[:, word_of(s, p_)] for p_ in range(bits)]
         for c in range(32):
             j = 32 * s + c
             if j >= cols:
@@ -195,10 +205,9 @@ def unpack_blob(blob: bytes):
     else:
         table = np.zeros((rows, G), np.uint16)
         zeros = np.zeros((rows, G), np.uint16)
-        zoff = (4 * S if bits == 3 else 5 * S) * 4
         for s in range(S):
-            pair = rec[:, 4 * s + 3] if bits == 3 else rec[:, 4 * S + s]
-            zb = rec.view(np.uint8)[:, zoff + s]
+            pair = rec[:, word_of(s, 3) if bits == 3 else 4 * S + s]
+            zb = rec.view(np.uint8)[:, zero_byte(s)]
             for e in range(2):
                 g = 2 * s + e
                 if g < G:
@@ -214,7 +223,8 @@ def unpack_blob(blob: bytes):
 
 
 @pytest.mark.parametrize("bits,mode,cols", [(3, "lut", 48), (4, "lut", 80), (3, "affine", 48),
-                                            (4, "affine", 112), (3, "affine", 1024), (3, "lut", 16)])
+                                            (4, "affine", 112), (3, "affine", 1024), (3, "lut", 16),
+                                            (3, "affine", 1040), (3, "affine", 2048 + 512 + 16)])
 def test_layout_round_trip(bits, mode, cols):
     p = synth.make_problem(7, cols, bits, mode, 0.03, "uniform", 2, 1)
     codes, table, zeros, rp, ci, va = unpack_blob(dsq.pack_problem(p))
