@@ -337,7 +337,9 @@ __device__ __forceinline__ void read_row(uint32_t rs, uint32_t rb, uint4 &v, uin
 // r0 + rg, r0 + rg + R, ...: each lane copies its slot's 16-byte record and
 // lanes 0, 1 the group's zero bytes, kD rows ahead, into the warp's ring
 // (cp.async, one commit group per row); each lane reads back its record and
-// zero byte.
+// zero byte.  A lane's wait covers only its own copies, so a warp barrier
+// follows each wait before the zero bytes are read; the refill of a stage
+// comes after the row's warp reduction, when every lane has read it.
 __global__ void __launch_bounds__(kThreads, 1)
 b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -394,7 +396,8 @@ b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y)
         for (; j + kD <= nj; j += kD) {
             unroll<0, kD>([&](auto dc) {
                 constexpr int d = decltype(dc)::value;
-                cp_async_wait<kD - 1>();  // row j + d has landed
+                cp_async_wait<kD - 1>();  // this lane's copies of row j + d have landed ...
+                __syncwarp();             // ... and every lane's (lanes 0, 1 copy the zero bytes)
                 uint4 v;
                 uint32_t zb;
                 read_row<d * kAffStageB>(rs, rb, v, zb);
@@ -408,6 +411,7 @@ b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y)
             });
         }
         cp_async_wait<0>();
+        __syncwarp();
         for (int d = 0; j < nj; j++, d++) {
             uint4 v;
             uint32_t zb;
