@@ -14,14 +14,18 @@
 //                the MMA reads (a deep ring; x is small and stays in L2);
 //   warp 1       allocates tensor memory, issues the MMAs (one thread), frees
 //                tensor memory;
-//   warps 2-17   decode: warp (quarter q = warp%4, slot half h, K-block
-//                parity kp) streams, for row 32q + lane, the 16-byte slot
-//                records and zero bytes of every second K-block straight from
-//                HBM (4 K-blocks ahead, double-buffered in registers), turns
-//                the 32 codes into 16 fp16 pairs -- LOP3 places two codes in
-//                the two halves of 1024.0, one HFMA2 gives the exact q - zero,
-//                one HMUL2 rounds scale*(q - zero) once -- and stores them into
-//                tensor memory (tcgen05.st) as the MMA's A operand;
+//   warp 22      record producer: per stage of 4 K-blocks, two 2-D TMA loads
+//                of the tile's packed rows -- 128 rows x 128 bytes of slot
+//                records (128-byte swizzle) and 128 rows x 16 bytes of their
+//                zero bytes -- into a ring of stages;
+//   warps 2-17   decode: warp (quarter q = warp%4, K-block j of the stage)
+//                reads, for row 32q + lane, its two slot records and zero
+//                bytes from the stage (conflict-free thanks to the swizzle),
+//                turns each slot's 32 codes into 16 fp16 pairs -- LOP3 places
+//                two codes in the two halves of 1024.0, one HFMA2 gives the
+//                exact q - zero, one HMUL2 rounds scale*(q - zero) once -- and
+//                stores them into tensor memory (tcgen05.st) as the MMA's A
+//                operand;
 //   warps 18-21  outliers: thread (row) walks its row's CSR entries that fall
 //                in each K-block and accumulates v * x[b][col] in fp32 from the
 //                staged x tile (exact products);
@@ -47,17 +51,30 @@ namespace {
 
 constexpr int kTM = 128;        // rows per tile (MMA M)
 constexpr int kKB = 64;         // columns per K-block (two slots)
-constexpr int kNA = 6;          // A stages in tensor memory
-constexpr int kU = 4;           // K-blocks a decode warp loads ahead
-constexpr int kWarps = 22;
+constexpr int kKS = 4;          // K-blocks per stage (8 slots: 128 bytes of each packed row)
+constexpr int kRecB = kTM * 128;                // record bytes of a stage
+constexpr int kStageRB = kRecB + kTM * 16;      // + the zero bytes (16 per row)
+constexpr int kWarps = 23;
 constexpr int kThreads = kWarps * 32;
-constexpr int kTmemCols = 256;  // accumulator at column 0, A stages from column 64
-constexpr int kACol0 = 64;
+constexpr int kTmemCols = 512;  // accumulators from column 0, then the A stages
 constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
 constexpr uint32_t kSentinel = 0xffffffffu;
 
+// Independent accumulators: consecutive MMAs into one accumulator serialise
+// on its latency, so MMA number n of the split goes to accumulator
+// n % NACC and the epilogue sums them.  Tensor memory: NACC accumulators of
+// NB columns, then NA stages of A (4 K-blocks = 128 columns each) -- 512
+// columns for every NB.
 template <int NB>
-__host__ __device__ constexpr int x_stages() { return NB <= 32 ? 12 : 8; }
+__host__ __device__ constexpr int n_acc() { return NB <= 32 ? 8 : 4; }
+template <int NB>
+__host__ __device__ constexpr int a_col0() { return NB * n_acc<NB>(); }
+template <int NB>
+__host__ __device__ constexpr int a_stages() { return (kTmemCols - a_col0<NB>()) / 128; }
+template <int NB>
+__host__ __device__ constexpr int x_stages() { return NB <= 32 ? 3 : 2; }  // of kKS x tiles
+template <int NB>
+__host__ __device__ constexpr int rec_stages() { return NB <= 32 ? 4 : 2; }
 
 struct TcParams {
     int rows, cols, S, row_words, nkb, kb_per_split, batch;
@@ -171,33 +188,37 @@ __device__ __forceinline__ int sw128_off(int b, int c) {
 }
 
 struct Smem {
-    uint64_t *afull, *aempty, *xfull, *xempty, *done;
+    uint64_t *afull, *aempty, *xfull, *xempty, *done, *rfull, *rempty;
     uint32_t *tmem_slot;
-    unsigned char *x;
+    unsigned char *x, *rec;
     float *obuf, *rbuf;
 };
 
 template <int NB>
 __device__ __forceinline__ Smem carve(unsigned char *base) {
-    constexpr int NX = x_stages<NB>();
+    constexpr int NX = x_stages<NB>(), NA = a_stages<NB>(), NR = rec_stages<NB>();
     Smem s;
     uint64_t *bars = reinterpret_cast<uint64_t *>(base);
     s.afull = bars;
-    s.aempty = bars + kNA;
-    s.xfull = bars + 2 * kNA;
-    s.xempty = bars + 2 * kNA + NX;
-    s.done = bars + 2 * kNA + 2 * NX;
-    s.tmem_slot = reinterpret_cast<uint32_t *>(s.done + 1);
-    s.x = base + 1024;
-    s.obuf = reinterpret_cast<float *>(s.x + NX * NB * 128);
+    s.aempty = s.afull + NA;
+    s.xfull = s.aempty + NA;
+    s.xempty = s.xfull + NX;
+    s.done = s.xempty + NX;
+    s.rfull = s.done + 1;
+    s.rempty = s.rfull + NR;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.rempty + NR);
+    s.x = base + 1024;                  // stages of kKS tiles [NB][64] fp16
+    s.rec = s.x + NX * kKS * NB * 128;  // stages of kStageRB bytes
+    s.obuf = reinterpret_cast<float *>(s.rec + NR * kStageRB);
     s.rbuf = s.obuf + kTM * NB;
     return s;
 }
 
-// 1 KB alignment slack + barriers + x ring + outlier sums + cluster inbox.
+// 1 KB alignment slack + barriers + x ring + record ring + outlier sums + cluster inbox.
 template <int NB>
 __host__ __device__ constexpr size_t smem_bytes(int KS) {
-    return 2048 + (size_t)x_stages<NB>() * NB * 128 + (size_t)kTM * NB * 4 * KS;
+    return 2048 + (size_t)x_stages<NB>() * kKS * NB * 128 + (size_t)rec_stages<NB>() * kStageRB +
+           (size_t)kTM * NB * 4 * KS;
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -216,27 +237,34 @@ __device__ __forceinline__ void st_cluster_f32(const float *local, uint32_t rank
 
 template <int NB>
 __global__ void __launch_bounds__(kThreads, 1)
-tc_kernel(const __grid_constant__ CUtensorMap tm_x, TcParams p, int KS, __half *__restrict__ y) {
+tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_rec,
+          const __grid_constant__ CUtensorMap tm_zero, TcParams p, int KS, __half *__restrict__ y) {
     static_assert(NB == 16 || NB == 32 || NB == 64, "NB");
-    constexpr int NX = x_stages<NB>();
+    constexpr int NX = x_stages<NB>(), NA = a_stages<NB>(), NR = rec_stages<NB>(), NACC = n_acc<NB>();
+    constexpr int XB = kKS * NB * 128;  // bytes of one x stage
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    // 1024-byte alignment for the swizzled x tiles (1 KB of slack is allocated)
+    // 1024-byte alignment for the swizzled tiles (1 KB of slack is allocated)
     unsigned char *smem_base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const Smem sm = carve<NB>(smem_base);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = KS > 1 ? (int)cluster_rank() : 0;
     const int tile = blockIdx.y;
-    const int kb0 = rank * p.kb_per_split;
+    const int kb0 = rank * p.kb_per_split;  // a multiple of kKS
     const int nk = max(0, min(p.nkb, kb0 + p.kb_per_split) - kb0);
+    const int t0 = kb0 / kKS, nst = (nk + kKS - 1) / kKS;  // stages of this split
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNA; i++) {
-            mbar_init(&sm.afull[i], 8);
+        for (int i = 0; i < NA; i++) {
+            mbar_init(&sm.afull[i], 16);  // every decode warp, once per stage
             mbar_init(&sm.aempty[i], 1);
+        }
+        for (int i = 0; i < NR; i++) {
+            mbar_init(&sm.rfull[i], 1);
+            mbar_init(&sm.rempty[i], 16);
         }
         for (int i = 0; i < NX; i++) {
             mbar_init(&sm.xfull[i], 1);
-            mbar_init(&sm.xempty[i], 1 + 4);
+            mbar_init(&sm.xempty[i], 1 + 4);  // the MMAs and the four outlier warps
         }
         mbar_init(sm.done, 1);
         fence_mbar_init();
@@ -253,94 +281,99 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, TcParams p, int KS, __half *
     const uint32_t tmem = *sm.tmem_slot;
 
     if (warp == 0) {
+        // x producer: per stage, the kKS x tiles [NB][64] (128-byte swizzle)
         if (lane == 0) {
             int issued = 0;
-            for (int i = 0; i < nk; i++) {
+            for (int i = 0; i < nst; i++) {
                 const int s = i % NX;
                 if (i >= NX && !mbar_wait(&sm.xempty[s], ((i / NX) - 1) & 1)) {
                     report(p.status, kStatusTimeout);
                     break;
                 }
-                mbar_arrive_expect_tx(&sm.xfull[s], (uint32_t)(NB * 128));
-                tma2d(sm.x + s * NB * 128, &tm_x, kKB * (kb0 + i), 0, &sm.xfull[s]);
+                mbar_arrive_expect_tx(&sm.xfull[s], (uint32_t)XB);
+                for (int kb = 0; kb < kKS; kb++)
+                    tma2d(sm.x + s * XB + kb * NB * 128, &tm_x, kKB * (kb0 + kKS * i + kb), 0, &sm.xfull[s]);
                 issued = i + 1;
             }
             for (int i = max(0, issued - NX); i < issued; i++)
                 if (!mbar_wait(&sm.xfull[i % NX], (i / NX) & 1)) report(p.status, kStatusTimeout);
         }
     } else if (warp == 1) {
+        // MMA issuer: per stage, 4 MMAs (K = 16 each) per K-block into rotating accumulators
         if (lane == 0) {
             const uint32_t idesc = idesc_f16(NB);
-            for (int i = 0; i < nk; i++) {
-                const int a = i % kNA, s = i % NX;
-                if (!mbar_wait(&sm.afull[a], (i / kNA) & 1) || !mbar_wait(&sm.xfull[s], (i / NX) & 1)) {
+            int n = 0;
+            for (int i = 0; i < nst; i++) {
+                const int as = i % NA, s = i % NX;
+                if (!mbar_wait(&sm.afull[as], (i / NA) & 1) || !mbar_wait(&sm.xfull[s], (i / NX) & 1)) {
                     report(p.status, kStatusTimeout);
                     break;
                 }
                 tc_fence_after();
-                const uint64_t bdesc = sw128_desc(sm.x + s * NB * 128);
+                for (int kb = 0; kb < kKS && kKS * i + kb < nk; kb++) {
+                    const uint64_t bdesc = sw128_desc(sm.x + s * XB + kb * NB * 128);
 #pragma unroll
-                for (int k = 0; k < 4; k++)
-                    tc_mma(tmem, tmem + kACol0 + 32 * a + 8 * k, bdesc + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
-                tc_commit(&sm.aempty[a]);
+                    for (int k = 0; k < 4; k++, n++)
+                        tc_mma(tmem + NB * (n % NACC), tmem + a_col0<NB>() + 128 * as + 32 * kb + 8 * k, bdesc + 2 * k,
+                               idesc, n >= NACC ? 1u : 0u);
+                }
+                tc_commit(&sm.aempty[as]);
                 tc_commit(&sm.xempty[s]);
             }
             tc_commit(sm.done);  // fires once every MMA issued above has completed
         }
     } else if (warp < 18) {
-        const int d = warp - 2;
-        const int q = warp & 3, h = (d >> 2) & 1, kp = d >> 3;
+        // decode: warp (quarter q, K-block j of every stage)
+        const int q = warp & 3, j = (warp - 2) >> 2;
         const int r = 32 * q + lane;
-        const int grow = kTM * tile + r;
         const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16);
-        const uint32_t *rec = p.dense + (size_t)min(grow, p.rows - 1) * p.row_words;
-        uint4 cur[kU], nxt[kU];
-        uint32_t czb[kU], nzb[kU];
-        // K-blocks of this warp: kp, kp + 2, ...; batch j holds the kU K-blocks kp + 2*(kU*j + u)
-        auto load = [&](int j, uint4 (&v)[kU], uint32_t (&zb)[kU]) {
-#pragma unroll
-            for (int u = 0; u < kU; u++) {
-                const int i = kp + 2 * (kU * j + u);
-                const int slot = 2 * (kb0 + i) + h;
-                v[u] = make_uint4(0u, 0u, 0u, 0u);
-                zb[u] = 0u;
-                if (i < nk && slot < p.S && grow < p.rows) {
-                    v[u] = __ldg(reinterpret_cast<const uint4 *>(rec + code_word_index(3, 1, p.S, slot, 0)));
-                    zb[u] = __ldg(reinterpret_cast<const uint8_t *>(rec) + zero_byte_index(3, p.S, slot));
-                }
+        for (int i = 0; i < nst; i++) {
+            const int st = i % NR, as = i % NA;
+            if (!mbar_wait_warp(&sm.rfull[st], (i / NR) & 1) ||
+                (i >= NA && !mbar_wait_warp(&sm.aempty[as], ((i / NA) - 1) & 1))) {
+                if (lane == 0) report(p.status, kStatusTimeout);
+                break;
             }
-        };
-        load(0, cur, czb);
-        bool ok = true;
-        for (int j = 0; ok && kp + 2 * kU * j < nk; j++) {
-            load(j + 1, nxt, nzb);
+            const int t = t0 + i;
+            if (kKS * i + j < nk) {
+                const unsigned char *rs = sm.rec + st * kStageRB;
+                tc_fence_after();
 #pragma unroll
-            for (int u = 0; u < kU; u++) {
-                const int i = kp + 2 * (kU * j + u);
-                if (i >= nk) break;  // warp-uniform
-                const int a = i % kNA;
-                if (i >= kNA && !mbar_wait_warp(&sm.aempty[a], ((i / kNA) - 1) & 1)) {
-                    if (lane == 0) report(p.status, kStatusTimeout);
-                    ok = false;
+                for (int h = 0; h < 2; h++) {
+                    const int c = 2 * j + h;  // 16-byte chunk of the row = slot of the stage
+                    const uint4 v = *reinterpret_cast<const uint4 *>(rs + r * 128 + ((c ^ (r & 7)) << 4));
+                    const uint32_t zb = rs[kRecB + r * 16 + 8 * (t & 1) + c];
+                    uint32_t o[16];
+                    decode_slot_f16(v, zb, o);  // records past the row's end read as 0 and decode to 0
+                    tc_st16(tbase + a_col0<NB>() + 128 * as + 32 * j + 16 * h, o);
+                }
+                tc_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.afull[as]);
+                mbar_arrive(&sm.rempty[st]);
+            }
+        }
+    } else if (warp == 22) {
+        // record producer
+        if (lane == 0) {
+            for (int i = 0; i < nst; i++) {
+                const int st = i % NR, t = t0 + i;
+                if (i >= NR && !mbar_wait(&sm.rempty[st], ((i / NR) - 1) & 1)) {
+                    report(p.status, kStatusTimeout);
                     break;
                 }
-                uint32_t o[16];
-                decode_slot_f16(cur[u], czb[u], o);  // zero records decode to 0 (scale 0)
-                tc_fence_after();
-                tc_st16(tbase + kACol0 + 32 * a + 16 * h, o);
-                tc_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.afull[a]);
-            }
-#pragma unroll
-            for (int u = 0; u < kU; u++) {
-                cur[u] = nxt[u];
-                czb[u] = nzb[u];
+                unsigned char *rs = sm.rec + st * kStageRB;
+                const int g = (2 * kKS * t) / 32, u = (2 * kKS * t) % 32;  // group, first slot in it
+                mbar_arrive_expect_tx(&sm.rfull[st], (uint32_t)kStageRB);
+                tma2d(rs, &tm_rec, kAff3GroupWords * g + 8 + 4 * u, kTM * tile, &sm.rfull[st]);
+                tma2d(rs + kRecB, &tm_zero, kAff3GroupWords * g + 4 * (u / 16), kTM * tile, &sm.rfull[st]);
             }
         }
     } else {
-        // outliers: thread = row
+        // outliers: thread = row, the entries in this split's columns, stage by stage
         const int r = 32 * (warp & 3) + lane;
         const int grow = kTM * tile + r;
         float acc[NB];
@@ -354,16 +387,19 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, TcParams p, int KS, __half *
         uint32_t qv[4];
 #pragma unroll
         for (int t = 0; t < 4; t++) qv[t] = k + t < kend ? __ldg(p.csr + k + t) : kSentinel;
-        for (int i = 0; i < nk; i++) {
+        const int cend = kKB * (kb0 + nk);  // first column past this split
+        for (int i = 0; i < nst; i++) {
             const int s = i % NX;
             if (!mbar_wait_warp(&sm.xfull[s], (i / NX) & 1)) {
                 if (lane == 0) report(p.status, kStatusTimeout);
                 break;
             }
-            const int c0 = kKB * (kb0 + i);
-            const unsigned char *xt = sm.x + s * NB * 128;
-            while ((int)(qv[0] & 0xffffu) < c0 + kKB) {
-                const int cl = (int)(qv[0] & 0xffffu) - c0;
+            const int c0 = kKB * (kb0 + kKS * i);
+            const int c1 = min(c0 + kKS * kKB, cend);
+            while ((int)(qv[0] & 0xffffu) < c1) {
+                const int cs = (int)(qv[0] & 0xffffu) - c0;
+                const unsigned char *xt = sm.x + s * XB + (cs >> 6) * NB * 128;
+                const int cl = cs & 63;
                 const unsigned short vb = (unsigned short)(qv[0] >> 16);
 #pragma unroll
                 for (int b = 0; b < NB; b++) {
@@ -397,12 +433,22 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, TcParams p, int KS, __half *
             have = false;
         }
         tc_fence_after();
+        // sum the accumulators that received MMAs (all of them once nk >= NACC/4)
+        const int nacc = min(4 * nk, n_acc<NB>());
 #pragma unroll
         for (int c = 0; c < NB; c += 16) {
             float v[16];
-            if (have) tc_ld16(tmem + ((uint32_t)(32 * q) << 16) + c, v);
 #pragma unroll
-            for (int t = 0; t < 16; t++) part[c + t] = (have ? v[t] : 0.f) + sm.obuf[r * NB + c + t];
+            for (int t = 0; t < 16; t++) v[t] = 0.f;
+            if (have)
+                for (int u = 0; u < nacc; u++) {
+                    float w[16];
+                    tc_ld16(tmem + ((uint32_t)(32 * q) << 16) + NB * u + c, w);
+#pragma unroll
+                    for (int t = 0; t < 16; t++) v[t] += w[t];
+                }
+#pragma unroll
+            for (int t = 0; t < 16; t++) part[c + t] = v[t] + sm.obuf[r * NB + c + t];
         }
         if (KS > 1 && rank > 0) {
 #pragma unroll
@@ -452,7 +498,8 @@ bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_
 }
 
 template <int NB>
-int launch_nb(const TcParams &p, int KS, const CUtensorMap &tx, __half *y, cudaStream_t st) {
+int launch_nb(const TcParams &p, int KS, const CUtensorMap &tx, const CUtensorMap &trec, const CUtensorMap &tzero,
+              __half *y, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(KS, (p.rows + kTM - 1) / kTM, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -465,13 +512,13 @@ int launch_nb(const TcParams &p, int KS, const CUtensorMap &tx, __half *y, cudaS
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tc_kernel<NB>, tx, p, KS, y) == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, tc_kernel<NB>, tx, trec, tzero, p, KS, y) == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
 }
 
 template <int NB>
 int set_attr() {
     return cudaFuncSetAttribute(tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_bytes<NB>(4)) == cudaSuccess
+                                (int)smem_bytes<NB>(2)) == cudaSuccess
                ? DSQ_OK
                : DSQ_ERR_CUDA;
 }
@@ -484,7 +531,8 @@ int set_attrs() {
 }
 
 // K split of a matrix: KS CTAs (one cluster) per 128-row tile, as many as fit
-// one CTA per SM, at most 4 and at most one per K-block.
+// one CTA per SM, at most 2; a split covers whole stages (kKS K-blocks) and
+// none is empty.
 struct Split {
     int KS, nkb, kb_per_split;
 };
@@ -492,10 +540,12 @@ Split plan_split(const MatrixView &m, int sm_count) {
     Split sp;
     const int tiles = (m.rows + kTM - 1) / kTM;
     sp.nkb = (m.slots + 1) / 2;
+    const int stages = (sp.nkb + kKS - 1) / kKS;
     sp.KS = 1;
-    for (int k = 2; k <= 4; k++)
-        if (tiles * k <= sm_count && k <= sp.nkb) sp.KS = k;
-    sp.kb_per_split = (sp.nkb + sp.KS - 1) / sp.KS;
+    for (int k = 2; k <= 2; k++)  // the cluster inbox holds one peer's tile
+        if (tiles * k <= sm_count && k <= stages) sp.KS = k;
+    sp.kb_per_split = kKS * ((stages + sp.KS - 1) / sp.KS);
+    sp.KS = (sp.nkb + sp.kb_per_split - 1) / sp.kb_per_split;
     return sp;
 }
 
@@ -510,9 +560,17 @@ int run_tc(const MatrixView &m, const Split &sp, const int32_t *split_start, int
     for (int b0 = 0; b0 < batch; b0 += 64) {
         const int nb = std::min(64, batch - b0);
         const int NB = nb <= 16 ? 16 : nb <= 32 ? 32 : 64;
-        CUtensorMap tx;
+        CUtensorMap tx, trec, tzero;
         if (!encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x + (size_t)b0 * m.cols, m.cols, nb,
                        (uint64_t)m.cols * 2, kKB, NB, CU_TENSOR_MAP_SWIZZLE_128B))
+            return DSQ_ERR_CUDA;
+        // the packed rows as [rows][row_words] u32: stage boxes of 32 words (records,
+        // 128-byte swizzle) and 4 words (zero bytes) by 128 rows; past the row end or
+        // the last row the loads fill zeros
+        if (!encode_2d(&trec, CU_TENSOR_MAP_DATA_TYPE_UINT32, m.dense, m.row_words, m.rows, (uint64_t)m.row_words * 4,
+                       32, kTM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_2d(&tzero, CU_TENSOR_MAP_DATA_TYPE_UINT32, m.dense, m.row_words, m.rows,
+                       (uint64_t)m.row_words * 4, 4, kTM, CU_TENSOR_MAP_SWIZZLE_NONE))
             return DSQ_ERR_CUDA;
         TcParams p;
         p.rows = m.rows;
@@ -529,9 +587,9 @@ int run_tc(const MatrixView &m, const Split &sp, const int32_t *split_start, int
         p.status = status;
         __half *yb = y + (size_t)b0 * m.rows;
         int rc;
-        if (NB == 16) rc = launch_nb<16>(p, sp.KS, tx, yb, st);
-        else if (NB == 32) rc = launch_nb<32>(p, sp.KS, tx, yb, st);
-        else rc = launch_nb<64>(p, sp.KS, tx, yb, st);
+        if (NB == 16) rc = launch_nb<16>(p, sp.KS, tx, trec, tzero, yb, st);
+        else if (NB == 32) rc = launch_nb<32>(p, sp.KS, tx, trec, tzero, yb, st);
+        else rc = launch_nb<64>(p, sp.KS, tx, trec, tzero, yb, st);
         if (rc != DSQ_OK) return rc;
     }
     return DSQ_OK;
