@@ -299,10 +299,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 if (!mbar_wait(&sm.xfull[i % NX], (i / NX) & 1)) report(p.status, kStatusTimeout);
         }
     } else if (warp == 1) {
-        // MMA issuer: per stage, 4 MMAs (K = 16 each) per K-block into rotating accumulators
+        // MMA issuer: per stage, 4 MMAs (K = 16 each) per K-block into rotating
+        // accumulators.  The issuing thread shares its scheduler with busy
+        // decode warps, so a full stage is one unrolled run of MMAs with
+        // compile-time offsets.
         if (lane == 0) {
             const uint32_t idesc = idesc_f16(NB);
-            int n = 0;
             for (int i = 0; i < nst; i++) {
                 const int as = i % NA, s = i % NX;
                 if (!mbar_wait(&sm.afull[as], (i / NA) & 1) || !mbar_wait(&sm.xfull[s], (i / NX) & 1)) {
@@ -310,12 +312,19 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                     break;
                 }
                 tc_fence_after();
-                for (int kb = 0; kb < kKS && kKS * i + kb < nk; kb++) {
-                    const uint64_t bdesc = sw128_desc(sm.x + s * XB + kb * NB * 128);
+                const uint32_t a0 = tmem + a_col0<NB>() + 128 * as;
+                const uint64_t b0 = sw128_desc(sm.x + s * XB);
+                const int nkb = min(kKS, nk - kKS * i);  // K-blocks of this stage
+                if (nkb == kKS && i > 0) {
 #pragma unroll
-                    for (int k = 0; k < 4; k++, n++)
-                        tc_mma(tmem + NB * (n % NACC), tmem + a_col0<NB>() + 128 * as + 32 * kb + 8 * k, bdesc + 2 * k,
-                               idesc, n >= NACC ? 1u : 0u);
+                    for (int m = 0; m < 4 * kKS; m++)  // m = 4 * kb + k
+                        tc_mma(tmem + NB * (m % NACC), a0 + 32 * (m / 4) + 8 * (m % 4),
+                               b0 + ((m / 4) * NB * 128 >> 4) + 2 * (m % 4), idesc, 1u);
+                } else {
+                    for (int m = 0; m < 4 * nkb; m++)
+                        tc_mma(tmem + NB * (m % NACC), a0 + 32 * (m / 4) + 8 * (m % 4),
+                               b0 + ((m / 4) * NB * 128 >> 4) + 2 * (m % 4), idesc,
+                               (i > 0 || m >= NACC) ? 1u : 0u);
                 }
                 tc_commit(&sm.aempty[as]);
                 tc_commit(&sm.xempty[s]);
