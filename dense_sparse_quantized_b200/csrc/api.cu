@@ -115,17 +115,25 @@ extern "C" int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void 
     if (!aligned16(x) || !aligned16(y)) return DSQ_ERR_INVALID_ARG;
     DeviceGuard guard(h->device);
     if (!guard.ok) return DSQ_ERR_CUDA;
-    int rc = launch_gemv_tc(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
-    if (rc == DSQ_ERR_UNSUPPORTED) rc = launch_gemv_fused(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
-    if (rc == DSQ_ERR_UNSUPPORTED)
-        rc = launch_gemv_generic(h, (const __half *)x, (__half *)y, batch, (cudaStream_t)stream);
+    const __half *xh = (const __half *)x;
+    __half *yh = (__half *)y;
+    const cudaStream_t st = (cudaStream_t)stream;
+    // tensor cores where they cover the shape and batch; else the tuned
+    // batch-1 kernel once per activation row; else the generic kernel
+    int rc = launch_gemv_tc(h, xh, yh, batch, st);
+    if (rc == DSQ_ERR_UNSUPPORTED && fused_launch_count(h, 1) > 0) {
+        rc = DSQ_OK;
+        for (int b = 0; b < batch && rc == DSQ_OK; b++)
+            rc = launch_gemv_fused(h, xh + (size_t)b * h->view.cols, yh + (size_t)b * h->view.rows, 1, st);
+    }
+    if (rc == DSQ_ERR_UNSUPPORTED) rc = launch_gemv_generic(h, xh, yh, batch, st);
     return rc;
 }
 
 extern "C" int dsq_gemv_launches(dsq_handle_t h, int batch) {
     if (!h || batch < 1) return -1;
     int n = tc_launch_count(h, batch);
-    if (n < 0) n = fused_launch_count(h, batch);
+    if (n < 0 && fused_launch_count(h, 1) > 0) n = batch * fused_launch_count(h, 1);
     return n >= 0 ? n : gemv_launch_count(h, batch);
 }
 

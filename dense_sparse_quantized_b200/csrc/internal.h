@@ -55,6 +55,7 @@ struct Schedule {
 struct TcPlan {
     bool ready = false;
     int KS = 1, nkb = 0, kb_per_split = 0;
+    int min_batch = 3;  // smallest batch sent to the tensor cores
     int32_t *split_start = nullptr;  // device, KS x rows (KS > 1)
 };
 

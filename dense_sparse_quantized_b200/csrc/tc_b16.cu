@@ -1,4 +1,4 @@
-// tc_b16.cu -- batch >= 16: dequantise to fp16, contract on the 5th-gen
+// tc_b16.cu -- batch >= 3: dequantise to fp16, contract on the 5th-gen
 // tensor cores (tcgen05, accumulator in tensor memory), outliers in fp32.
 //
 // At 16+ activation rows the product is a real (skinny) GEMM, so the dense
@@ -606,7 +606,15 @@ int run_tc(const MatrixView &m, const Split &sp, const int32_t *split_start, int
 
 }  // namespace
 
-bool tc_covers(const dsq_handle_s *h, int batch) { return h->tc.ready && batch >= 16 && tc_shape_ok(h->view); }
+// From 3 activation rows on, one tensor-core pass (the batch padded to 16
+// with zero rows by the x loads) beats the batch-1 kernel run per row --
+// unless a row carries hundreds of outliers: the outlier warps walk one row
+// per thread, so such matrices go to the tensor cores from 16 rows on.
+constexpr int kTcMinBatch = 3, kTcMinBatchHeavy = 16, kHeavyRowNnz = 256;
+
+bool tc_covers(const dsq_handle_s *h, int batch) {
+    return h->tc.ready && batch >= h->tc.min_batch && tc_shape_ok(h->view);
+}
 
 int tc_launch_count(const dsq_handle_s *h, int batch) { return tc_covers(h, batch) ? (batch + 63) / 64 : -1; }
 
@@ -623,6 +631,9 @@ int tc_prepare(dsq_handle_s *h, const int32_t *rp, const uint32_t *csr_host) {
     tc.KS = KS;
     tc.nkb = sp.nkb;
     tc.kb_per_split = sp.kb_per_split;
+    int max_nnz = 0;
+    for (int r = 0; r < m.rows; r++) max_nnz = std::max(max_nnz, rp[r + 1] - rp[r]);
+    tc.min_batch = max_nnz > kHeavyRowNnz ? kTcMinBatchHeavy : kTcMinBatch;
     if (KS > 1) {
         std::vector<int32_t> starts((size_t)KS * m.rows);
         for (int s = 0; s < KS; s++) {
