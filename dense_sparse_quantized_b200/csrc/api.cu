@@ -121,6 +121,7 @@ extern "C" int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void 
     // tensor cores where they cover the shape and batch; else the tuned
     // batch-1 kernel once per activation row; else the generic kernel
     int rc = launch_gemv_tc(h, xh, yh, batch, st);
+    if (rc == DSQ_ERR_UNSUPPORTED && batch > 1) rc = launch_gemv_batched(h, xh, yh, batch, st);
     if (rc == DSQ_ERR_UNSUPPORTED && fused_launch_count(h, 1) > 0) {
         rc = DSQ_OK;
         for (int b = 0; b < batch && rc == DSQ_OK; b++)
@@ -133,6 +134,7 @@ extern "C" int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void 
 extern "C" int dsq_gemv_launches(dsq_handle_t h, int batch) {
     if (!h || batch < 1) return -1;
     int n = tc_launch_count(h, batch);
+    if (n < 0 && batch > 1) n = batched_launch_count(h, batch);
     if (n < 0 && fused_launch_count(h, 1) > 0) n = batch * fused_launch_count(h, 1);
     return n >= 0 ? n : gemv_launch_count(h, batch);
 }

@@ -524,6 +524,231 @@ b1_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) 
     finalize(td, smem, p, 1.0f, y);
 }
 
+// ---------------------------------------------------------------- small batches
+
+constexpr int kMaxWarpsN = 12;  // batched table kernel: fewer warps, room for x of 4 rows in registers
+constexpr int kThreadsN = kMaxWarpsN * 32;
+
+// v[0..NB-1] (one value per activation row) summed over the warp in one
+// transposed butterfly; afterwards lane l holds the total of activation row
+// bn_row<NB>(l), in a fixed order.
+template <int NB>
+__device__ __forceinline__ float reduce_rows(float (&v)[NB], int lane) {
+    int o = 16;
+#pragma unroll
+    for (int n = NB; n > 1; n >>= 1, o >>= 1) {
+        const bool hi = lane & o;
+#pragma unroll
+        for (int i = 0; i < n / 2; i++) {
+            const float send = hi ? v[i] : v[i + n / 2], keep = hi ? v[i + n / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+    }
+#pragma unroll
+    for (; o >= 1; o >>= 1) v[0] += __shfl_xor_sync(kFull, v[0], o);
+    return v[0];
+}
+// The row whose total reduce_rows leaves in lane l: the halvings at lane
+// bits 4, 3, 2 pick it, high bit first; lanes with the remaining low bits
+// zero store it.
+template <int NB>
+__device__ __forceinline__ int bn_row(int lane) {
+    return NB == 8 ? (lane >> 2) & 7 : NB == 4 ? (lane >> 3) & 3 : (lane >> 4) & 1;
+}
+template <int NB>
+__device__ __forceinline__ bool bn_store_lane(int lane) {
+    return (lane & (NB == 8 ? 3 : NB == 4 ? 7 : 15)) == 0;
+}
+
+// Table rows, NB activation rows at once (NB = 2 or 4; nb <= NB real).
+// As the batch-1 table kernel, but each lane keeps its 32 columns of x for
+// every activation row as fp16 pairs, looks each weight up once (shfl.idx,
+// fp16 centroid) and adds weight * x for every row with mixed-precision
+// FMAs.  Outliers: one lane per piece after the dense loop, x read from L2.
+template <int BITS, int NB>
+__global__ void __launch_bounds__(kThreadsN, 1)
+bn_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y, int nb) {
+    constexpr int K = 1 << BITS;
+    constexpr int NW = BITS;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const MatrixView &m = p.m;
+    const int S = m.slots, C = p.C, R = p.R, N = m.cols;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const TileDesc td = p.tiles[blockIdx.x];
+    const int nrows = td.r1 - td.r0;
+    const int cw = warp % C, rg = warp / C;
+    const int s = cw * 32 + lane;
+    const bool valid = s < S;
+
+    const uint32_t ring = smem_u32(smem + p.off_ring + (size_t)warp * kDepth * kStageB);
+    const uint32_t ring_s = ring + 16 * lane, ring_a = ring + 512 + 4 * lane;
+    const size_t row_step = (size_t)R * m.row_words * 4;
+    const unsigned char *rec = reinterpret_cast<const unsigned char *>(m.dense) +
+                               ((size_t)td.r0 + rg) * m.row_words * 4;
+    const unsigned char *tabp = reinterpret_cast<const unsigned char *>(m.table) +
+                                ((size_t)(td.r0 + rg) * K + (lane & (K - 1))) * 2 - 2 * (lane & 1);
+    const int nj = rg < nrows ? (nrows - rg + R - 1) / R : 0;
+    int issued = 0;
+    auto issue = [&](int d) {
+        if (issued < nj) {
+            const uint32_t st = ring_s + d * kStageB, sa = ring_a + d * kStageB;
+            if (valid) {
+                if (NW == 4) {
+                    cp_async16(st, rec + 16 * s);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < NW; k++) cp_async4(st + 4 * k, rec + 4 * ((size_t)k * S + s));
+                }
+            }
+            cp_async4(sa, tabp);
+            rec += row_step;
+            tabp += (size_t)R * K * 2;
+        }
+        issued++;
+        cp_async_commit();
+    };
+    if (threadIdx.x == 0) {
+        mbar_init(reinterpret_cast<uint64_t *>(smem + kBarCsr), 1);
+        fence_mbar_init();
+        issue_csr(p, td, smem);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int d = 0; d < kDepth; d++) issue(d);
+
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // x of every activation row: this lane's 32 columns as fp16 pairs (rows past nb read 0)
+    uint32_t xh[NB][16];
+#pragma unroll
+    for (int b = 0; b < NB; b++) {
+        if (b < nb) {
+            x_pairs(x + (size_t)b * N, s, N, xh[b]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; i++) xh[b][i] = 0u;
+        }
+    }
+    float *part = reinterpret_cast<float *>(smem + p.off_part);  // [row][C][NB]
+    int i = rg;
+    for (int j = 0; j < nj; j++, i += R) {
+        const int d = j & (kDepth - 1);
+        cp_async_wait<kDepth - 1>();
+        const uint32_t st = ring_s + d * kStageB, sa = ring_a + d * kStageB;
+        uint32_t w4[4] = {0u, 0u, 0u, 0u};
+        if (valid) {
+            if (NW == 4) {
+                const uint4 q = lds128(st);
+                w4[0] = q.x; w4[1] = q.y; w4[2] = q.z; w4[3] = q.w;
+            } else {
+#pragma unroll
+                for (int k = 0; k < NW; k++) w4[k] = lds32(st + 4 * k);
+            }
+        }
+        // this lane's centroid as fp16 bits (the word holds two entries)
+        const uint32_t tv = (lds32(sa) >> (16 * (lane & 1))) & 0xffffu;
+        float lo[NB], hi[NB];
+#pragma unroll
+        for (int b = 0; b < NB; b++) lo[b] = hi[b] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+            int q0, q1;
+            if (BITS == 4) {
+                q0 = (int)(w4[c >> 3] >> (4 * (c & 7)));
+                q1 = (int)(w4[c >> 3] >> (4 * ((c + 1) & 7)));
+            } else if (c < 30) {
+                q0 = (int)(w4[c / 10] >> raw_pos3(c));
+                q1 = (int)(w4[(c + 1) / 10] >> raw_pos3(c + 1));
+            } else {
+                q0 = (int)(((w4[0] >> 9) & 1u) | ((w4[1] >> 8) & 2u) | ((w4[2] >> 7) & 4u));
+                q1 = (int)(((w4[0] >> 25) & 1u) | ((w4[1] >> 24) & 2u) | ((w4[2] >> 23) & 4u));
+            }
+            // shfl.idx over a 2^b-lane segment reads only the low b bits of the index
+            const uint32_t w0 = __shfl_sync(kFull, tv, q0, K), w1 = __shfl_sync(kFull, tv, q1, K);
+            const uint32_t wp = w0 | (w1 << 16);  // fp16 pair (column c, c + 1)
+#pragma unroll
+            for (int b = 0; b < NB; b++) mfma_pair(lo[b], hi[b], wp, xh[b][c >> 1]);
+        }
+        float v[NB];
+#pragma unroll
+        for (int b = 0; b < NB; b++) v[b] = lo[b] + hi[b];
+        const float t = reduce_rows<NB>(v, lane);
+        if (bn_store_lane<NB>(lane)) part[((size_t)i * C + cw) * NB + bn_row<NB>(lane)] = t;
+        issue(d);
+    }
+    cp_async_wait<0>();
+
+    // outliers: thread t sums pieces t, t + blockDim, ... for every activation row
+    if (wait_stage(smem, kBarCsr, p)) {
+        const uint32_t *csr = reinterpret_cast<const uint32_t *>(smem + p.off_csr);
+        const int32_t *pk = reinterpret_cast<const int32_t *>(smem + p.off_pk);
+        float *psum = reinterpret_cast<float *>(smem + p.off_psum);  // [piece][NB]
+        const int ka = td.k0 & ~3, pa = td.p0 & ~3;
+        for (int q = td.p0 + threadIdx.x; q < td.p1; q += blockDim.x) {
+            float a[NB];
+#pragma unroll
+            for (int b = 0; b < NB; b++) a[b] = 0.f;
+            for (int k = pk[q - pa] - ka; k < pk[q + 1 - pa] - ka; k++) {
+                const uint32_t e = csr[k];
+                const uint16_t v = (uint16_t)(e >> 16);
+                const int col = (int)(e & 0xffffu);
+#pragma unroll
+                for (int b = 0; b < NB; b++)
+                    if (b < nb) a[b] = mfma(v, __ldg(reinterpret_cast<const uint16_t *>(x) + (size_t)b * N + col), a[b]);
+            }
+#pragma unroll
+            for (int b = 0; b < NB; b++) psum[(size_t)(q - td.p0) * NB + b] = a[b];
+        }
+    }
+    __syncthreads();
+
+    // y[b][r] = sum_c part + the row's piece sums, in a fixed order: a lane per
+    // row, or the whole warp for a row with many pieces
+    const float *psum = reinterpret_cast<const float *>(smem + p.off_psum);
+    const int32_t *rp = reinterpret_cast<const int32_t *>(smem + p.off_rp);
+    const int ra = td.r0 & ~3, nw = blockDim.x >> 5;
+    for (int i0 = 32 * warp; i0 < nrows; i0 += 32 * nw) {
+        const int r = i0 + lane;
+        int q0 = 0, q1 = 0;
+        if (r < nrows) {
+            q0 = rp[td.r0 + r - ra];
+            q1 = rp[td.r0 + r + 1 - ra];
+        }
+        const bool heavy = q1 - q0 > kHeavyPieces;
+        float o[NB];
+#pragma unroll
+        for (int b = 0; b < NB; b++) {
+            o[b] = 0.f;
+            if (!heavy)
+                for (int q = q0; q < q1; q++) o[b] += psum[(size_t)(q - td.p0) * NB + b];
+        }
+        unsigned hm = __ballot_sync(kFull, heavy);
+        while (hm) {
+            const int src = __ffs(hm) - 1;
+            hm &= hm - 1;
+            const int h0 = __shfl_sync(kFull, q0, src), h1 = __shfl_sync(kFull, q1, src);
+#pragma unroll
+            for (int b = 0; b < NB; b++) {
+                float tsum = 0.f;
+                for (int q = h0 + lane; q < h1; q += 32) tsum += psum[(size_t)(q - td.p0) * NB + b];
+                tsum = warp_sum(tsum);
+                if (lane == src) o[b] = tsum;
+            }
+        }
+        if (r < nrows) {
+#pragma unroll
+            for (int b = 0; b < NB; b++) {
+                if (b < nb) {
+                    float acc = 0.f;
+                    for (int c = 0; c < C; c++) acc += part[((size_t)r * C + c) * NB + b];
+                    y[(size_t)b * m.rows + td.r0 + r] = __float2half_rn(acc + o[b]);
+                }
+            }
+        }
+    }
+}
+
 enum Kind { kNone = -1, kAff3 = 0, kLut3 = 3, kLut4 = 4 };
 
 Kind b1_kind(const MatrixView &m, int batch) {
@@ -592,6 +817,39 @@ int upload(T **dst, const std::vector<T> &v, size_t pad_elems, size_t *acct) {
     return DSQ_OK;
 }
 
+// Launch geometry and shared-memory map of the batched table kernel.
+bool plan_bn(const dsq_handle_s *h, int NB, B1Params *out, size_t *smem_bytes) {
+    const MatrixView &m = h->view;
+    const Schedule &sc = h->sched;
+    B1Params p;
+    p.m = m;
+    p.tiles = sc.tiles;
+    p.row_piece = sc.row_piece;
+    p.piece_k = sc.piece_k;
+    p.status = h->d_status;
+    p.C = (m.slots + 31) / 32;
+    p.R = std::max(1, kMaxWarpsN / p.C);
+    if (p.C > kMaxWarpsN) return false;
+    size_t off = 128;  // mbarrier
+    p.off_x = (int)off;  // unused
+    p.off_csr = (int)off;
+    off = align_sz(off + (size_t)(sc.max_csr + 8) * 4, 16);
+    p.off_rp = (int)off;
+    off = align_sz(off + (size_t)(sc.max_rows + 9) * 4, 16);
+    p.off_pk = (int)off;
+    off = align_sz(off + (size_t)(sc.max_pieces + 9) * 4, 16);
+    p.off_part = (int)off;
+    off = align_sz(off + (size_t)sc.max_rows * p.C * NB * 4, 16);
+    p.off_psum = (int)off;
+    off = align_sz(off + (size_t)(sc.max_pieces + 1) * NB * 4, 128);
+    p.off_ring = (int)off;
+    off += (size_t)p.C * p.R * kDepth * kStageB;
+    if (off > kSmemBudget) return false;
+    *out = p;
+    *smem_bytes = off;
+    return true;
+}
+
 }  // namespace
 
 // Row tiles of about equal cost (record bytes + a per-outlier charge), each
@@ -657,7 +915,57 @@ int fused_prepare(dsq_handle_s *) {
     int rc = set_smem_attr(b1_aff3_kernel);
     if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<kLut3>);
     if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<kLut4>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<3, 2>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<3, 4>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<4, 2>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<4, 4>);
     return rc;
+}
+
+// Table matrices at batch >= 2: chunks of 4 activation rows, each one
+// launch of the batched kernel (2 or 4 rows wide; 8 rows of x in registers
+// left too few warps per SM and measured slower than two passes of 4).
+int batched_launch_count(const dsq_handle_s *h, int batch) {
+    B1Params p;
+    size_t smem;
+    const MatrixView &m = h->view;
+    if (batch < 2 || m.mode != DSQ_MODE_LUT_ROW || m.rows <= 0 || m.cols <= 0 || h->sched.n_tiles == 0 ||
+        !plan_bn(h, 4, &p, &smem))
+        return -1;
+    return (batch + 3) / 4;
+}
+
+int launch_gemv_batched(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t st) {
+    if (batched_launch_count(h, batch) < 0) return DSQ_ERR_UNSUPPORTED;
+    const MatrixView &m = h->view;
+    for (int b0 = 0; b0 < batch; b0 += 4) {
+        const int nb = std::min(4, batch - b0);
+        const int NB = nb <= 2 ? 2 : 4;
+        B1Params p;
+        size_t smem;
+        if (!plan_bn(h, NB, &p, &smem)) return DSQ_ERR_UNSUPPORTED;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(h->sched.n_tiles, 1, 1);
+        cfg.blockDim = dim3(p.C * p.R * 32, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const __half *xb = x + (size_t)b0 * m.cols;
+        __half *yb = y + (size_t)b0 * m.rows;
+        cudaError_t e;
+        if (m.bits == 3)
+            e = NB == 2 ? cudaLaunchKernelEx(&cfg, bn_lut_kernel<3, 2>, p, xb, yb, nb)
+                        : cudaLaunchKernelEx(&cfg, bn_lut_kernel<3, 4>, p, xb, yb, nb);
+        else
+            e = NB == 2 ? cudaLaunchKernelEx(&cfg, bn_lut_kernel<4, 2>, p, xb, yb, nb)
+                        : cudaLaunchKernelEx(&cfg, bn_lut_kernel<4, 4>, p, xb, yb, nb);
+        if (e != cudaSuccess) return DSQ_ERR_CUDA;
+    }
+    return DSQ_OK;
 }
 
 int fused_launch_count(const dsq_handle_s *h, int batch) {

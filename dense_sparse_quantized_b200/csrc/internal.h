@@ -90,6 +90,9 @@ void free_schedule(dsq_handle_s *h);
 int fused_prepare(dsq_handle_s *h);
 int fused_launch_count(const dsq_handle_s *h, int batch);
 int launch_gemv_fused(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
+// Table matrices at batch >= 2 (fused_b1.cu), same convention.
+int batched_launch_count(const dsq_handle_s *h, int batch);
+int launch_gemv_batched(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
 
 // Tensor-core path (tc_b16.cu), same convention.
 int tc_prepare(dsq_handle_s *h, const int32_t *row_ptr_host, const uint32_t *csr_host);
