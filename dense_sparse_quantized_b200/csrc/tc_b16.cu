@@ -75,6 +75,11 @@ template <int NB>
 __host__ __device__ constexpr int x_stages() { return NB <= 32 ? 3 : 2; }  // of kKS x tiles
 template <int NB>
 __host__ __device__ constexpr int rec_stages() { return NB <= 32 ? 4 : 2; }
+// Shared memory for the tile's CSR entries (all of its rows, every split),
+// staged by one bulk copy; a tile with more entries reads them from global
+// memory, one row per thread.
+template <int NB>
+__host__ __device__ constexpr int csr_cap_bytes() { return NB == 16 ? 96 * 1024 : NB == 32 ? 64 * 1024 : 56 * 1024; }
 
 struct TcParams {
     int rows, cols, S, row_words, nkb, kb_per_split, batch;
@@ -188,10 +193,11 @@ __device__ __forceinline__ int sw128_off(int b, int c) {
 }
 
 struct Smem {
-    uint64_t *afull, *aempty, *xfull, *xempty, *done, *rfull, *rempty;
+    uint64_t *afull, *aempty, *xfull, *xempty, *done, *rfull, *rempty, *csrfull;
     uint32_t *tmem_slot;
     unsigned char *x, *rec;
     float *obuf, *rbuf;
+    uint32_t *csr;
 };
 
 template <int NB>
@@ -206,20 +212,25 @@ __device__ __forceinline__ Smem carve(unsigned char *base) {
     s.done = s.xempty + NX;
     s.rfull = s.done + 1;
     s.rempty = s.rfull + NR;
-    s.tmem_slot = reinterpret_cast<uint32_t *>(s.rempty + NR);
+    s.csrfull = s.rempty + NR;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.csrfull + 1);
     s.x = base + 1024;                  // stages of kKS tiles [NB][64] fp16
     s.rec = s.x + NX * kKS * NB * 128;  // stages of kStageRB bytes
     s.obuf = reinterpret_cast<float *>(s.rec + NR * kStageRB);
     s.rbuf = s.obuf + kTM * NB;
+    s.csr = reinterpret_cast<uint32_t *>(s.rbuf + kTM * NB);
     return s;
 }
 
-// 1 KB alignment slack + barriers + x ring + record ring + outlier sums + cluster inbox.
+// 1 KB alignment slack + barriers + x ring + record ring + outlier sums +
+// cluster inbox + staged CSR entries.
 template <int NB>
-__host__ __device__ constexpr size_t smem_bytes(int KS) {
+__host__ __device__ constexpr size_t smem_bytes() {
     return 2048 + (size_t)x_stages<NB>() * kKS * NB * 128 + (size_t)rec_stages<NB>() * kStageRB +
-           (size_t)kTM * NB * 4 * KS;
+           (size_t)kTM * NB * 4 * 2 + csr_cap_bytes<NB>();
 }
+static_assert(smem_bytes<16>() <= 232448 && smem_bytes<32>() <= 232448 && smem_bytes<64>() <= 232448,
+              "shared memory per CTA");
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -267,6 +278,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             mbar_init(&sm.xempty[i], 1 + 4);  // the MMAs and the four outlier warps
         }
         mbar_init(sm.done, 1);
+        mbar_init(sm.csrfull, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -388,14 +400,29 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
         float acc[NB];
 #pragma unroll
         for (int b = 0; b < NB; b++) acc[b] = 0.f;
+        // the tile's entries [ka, kz), rounded out to 16 bytes (the blob is padded past the end)
+        const int ka = __ldg(p.row_ptr + kTM * tile) & ~3;
+        const int kz = (__ldg(p.row_ptr + min(kTM * tile + kTM, p.rows)) + 3) & ~3;
+        const bool staged = kz > ka && (kz - ka) * 4 <= csr_cap_bytes<NB>();
+        if (staged && warp == 18 && lane == 0) {
+            mbar_arrive_expect_tx(sm.csrfull, (uint32_t)(kz - ka) * 4);
+            bulk_g2s(sm.csr, p.csr + ka, (uint32_t)(kz - ka) * 4, sm.csrfull);
+        }
         int k = 0, kend = 0;
         if (grow < p.rows && nk > 0) {
             k = p.split_start ? p.split_start[(size_t)rank * p.rows + grow] : p.row_ptr[grow];
             kend = p.row_ptr[grow + 1];
         }
+        if (staged && !mbar_wait_warp(sm.csrfull, 0)) {
+            if (lane == 0) report(p.status, kStatusTimeout);
+            kend = k;  // the entries never arrived: none are read
+        }
+        auto entry = [&](int e) -> uint32_t {
+            return e < kend ? (staged ? sm.csr[e - ka] : __ldg(p.csr + e)) : kSentinel;
+        };
         uint32_t qv[4];
 #pragma unroll
-        for (int t = 0; t < 4; t++) qv[t] = k + t < kend ? __ldg(p.csr + k + t) : kSentinel;
+        for (int t = 0; t < 4; t++) qv[t] = entry(k + t);
         const int cend = kKB * (kb0 + nk);  // first column past this split
         for (int i = 0; i < nst; i++) {
             const int s = i % NX;
@@ -419,7 +446,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
                 qv[1] = qv[2];
                 qv[2] = qv[3];
                 k++;
-                qv[3] = k + 3 < kend ? __ldg(p.csr + k + 3) : kSentinel;
+                qv[3] = entry(k + 3);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.xempty[s]);
@@ -512,7 +539,7 @@ int launch_nb(const TcParams &p, int KS, const CUtensorMap &tx, const CUtensorMa
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(KS, (p.rows + kTM - 1) / kTM, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem_bytes<NB>(KS);
+    cfg.dynamicSmemBytes = smem_bytes<NB>();
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -527,7 +554,7 @@ int launch_nb(const TcParams &p, int KS, const CUtensorMap &tx, const CUtensorMa
 template <int NB>
 int set_attr() {
     return cudaFuncSetAttribute(tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_bytes<NB>(2)) == cudaSuccess
+                                (int)smem_bytes<NB>()) == cudaSuccess
                ? DSQ_OK
                : DSQ_ERR_CUDA;
 }

@@ -172,6 +172,30 @@ def test_all_outlier_rows(orc, mode):
         check_y(gemv(h, q.x, 2), y_ref, bound, "all-outlier rows")
 
 
+@pytest.mark.parametrize("batch", [16, 40])
+def test_tile_outliers_staged_and_not(orc, batch):
+    """Tensor-core path: the first 128-row tile holds 300 outliers per row, more
+    than the CSR slice kept in shared memory, so its outlier warps read the
+    entries from global memory; the other tiles (the last one ragged) are
+    staged.  Both must match the oracle."""
+    p = synth.make_problem(300, 2048, 3, "affine", 0.01, "uniform", 77, batch)
+    rng = np.random.default_rng(2)
+    rows = []
+    for i in range(p.rows):
+        if i < 128:
+            rows.append(np.sort(rng.choice(p.cols, 300, replace=False)))
+        else:
+            rows.append(p.col_idx[p.row_ptr[i]:p.row_ptr[i + 1]])
+    counts = np.array([len(r) for r in rows])
+    rp = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    ci = np.concatenate(rows).astype(np.int32)
+    va = synth.f16_bits(rng.laplace(0, 0.2, ci.size))
+    q = edited(p, row_ptr=rp, col_idx=ci, values=va)
+    with dsq.Handle(dsq.pack_problem(q)) as h:
+        y_ref, bound = orc.gemv(q)
+        check_y(gemv(h, q.x, batch), y_ref, bound, f"staged and unstaged tiles B={batch}")
+
+
 @pytest.mark.parametrize("name", ["c2", "c3"])
 def test_zero_and_one_hot_x(orc, name):
     p, h = config(name)
