@@ -42,6 +42,7 @@ struct TileDesc {
 constexpr int kPieceMax = 31;
 struct Schedule {
     int n_tiles = 0;
+    int per_sm = 1;       // CTAs per SM the tiles were cut for (batch-1 affine kernel)
     int max_rows = 0;     // rows of the largest tile
     int max_pieces = 0;   // pieces of the largest tile
     int max_csr = 0;      // CSR entries of the largest tile
