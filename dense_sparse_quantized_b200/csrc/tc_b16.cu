@@ -79,7 +79,17 @@ __host__ __device__ constexpr int rec_stages() { return NB <= 32 ? 4 : 2; }
 // staged by one bulk copy; a tile with more entries reads them from global
 // memory, one row per thread.
 template <int NB>
-__host__ __device__ constexpr int csr_cap_bytes() { return NB == 16 ? 96 * 1024 : NB == 32 ? 64 * 1024 : 56 * 1024; }
+__host__ __device__ constexpr int csr_cap_bytes() { return NB == 16 ? 96 * 1024 : NB == 32 ? 64 * 1024 : 24 * 1024; }
+// At 64 activation rows the outlier warps first copy each x stage
+// column-major (the NB values of one column NB * 2 contiguous bytes) and read
+// an entry's x values with NB / 8 16-byte loads instead of NB 2-byte loads
+// from the swizzled tiles.  At 16 and 32 rows the copy and its two extra
+// synchronisations per stage cost more than they save (measured: c4 q at 32
+// rows 34.7 us without, 48.7 us with; at 64 rows 117 us without, 103 us with).
+template <int NB>
+__host__ __device__ constexpr bool col_major_x() { return NB >= 64; }
+template <int NB>
+__host__ __device__ constexpr int xt_bytes() { return col_major_x<NB>() ? kKS * kKB * NB * 2 : 0; }
 
 struct TcParams {
     int rows, cols, S, row_words, nkb, kb_per_split, batch;
@@ -193,9 +203,9 @@ __device__ __forceinline__ int sw128_off(int b, int c) {
 }
 
 struct Smem {
-    uint64_t *afull, *aempty, *xfull, *xempty, *done, *rfull, *rempty, *csrfull;
+    uint64_t *afull, *aempty, *xfull, *xempty, *done, *rfull, *rempty, *csrfull, *xtready, *xtfree;
     uint32_t *tmem_slot;
-    unsigned char *x, *rec;
+    unsigned char *x, *rec, *xt;
     float *obuf, *rbuf;
     uint32_t *csr;
 };
@@ -213,21 +223,24 @@ __device__ __forceinline__ Smem carve(unsigned char *base) {
     s.rfull = s.done + 1;
     s.rempty = s.rfull + NR;
     s.csrfull = s.rempty + NR;
-    s.tmem_slot = reinterpret_cast<uint32_t *>(s.csrfull + 1);
+    s.xtready = s.csrfull + 1;
+    s.xtfree = s.xtready + 1;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.xtfree + 1);
     s.x = base + 1024;                  // stages of kKS tiles [NB][64] fp16
     s.rec = s.x + NX * kKS * NB * 128;  // stages of kStageRB bytes
     s.obuf = reinterpret_cast<float *>(s.rec + NR * kStageRB);
     s.rbuf = s.obuf + kTM * NB;
     s.csr = reinterpret_cast<uint32_t *>(s.rbuf + kTM * NB);
+    s.xt = reinterpret_cast<unsigned char *>(s.csr) + csr_cap_bytes<NB>();
     return s;
 }
 
 // 1 KB alignment slack + barriers + x ring + record ring + outlier sums +
-// cluster inbox + staged CSR entries.
+// cluster inbox + staged CSR entries + column-major x stage.
 template <int NB>
 __host__ __device__ constexpr size_t smem_bytes() {
     return 2048 + (size_t)x_stages<NB>() * kKS * NB * 128 + (size_t)rec_stages<NB>() * kStageRB +
-           (size_t)kTM * NB * 4 * 2 + csr_cap_bytes<NB>();
+           (size_t)kTM * NB * 4 * 2 + csr_cap_bytes<NB>() + xt_bytes<NB>();
 }
 static_assert(smem_bytes<16>() <= 232448 && smem_bytes<32>() <= 232448 && smem_bytes<64>() <= 232448,
               "shared memory per CTA");
@@ -275,10 +288,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
         }
         for (int i = 0; i < NX; i++) {
             mbar_init(&sm.xfull[i], 1);
-            mbar_init(&sm.xempty[i], 1 + 4);  // the MMAs and the four outlier warps
+            mbar_init(&sm.xempty[i], 1 + 4);  // the MMAs and the four outlier warps (after their transpose)
         }
         mbar_init(sm.done, 1);
         mbar_init(sm.csrfull, 1);
+        mbar_init(sm.xtready, 4);  // the four outlier warps, once per stage
+        mbar_init(sm.xtfree, 4);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -424,7 +439,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
 #pragma unroll
         for (int t = 0; t < 4; t++) qv[t] = entry(k + t);
         const int cend = kKB * (kb0 + nk);  // first column past this split
-        for (int i = 0; i < nst; i++) {
+        for (int i = 0; i < nst && !col_major_x<NB>(); i++) {
             const int s = i % NX;
             if (!mbar_wait_warp(&sm.xfull[s], (i / NX) & 1)) {
                 if (lane == 0) report(p.status, kStatusTimeout);
@@ -450,6 +465,71 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.xempty[s]);
+        }
+        // column pair of the stage this thread transposes: K-block kt, columns 2 jp, 2 jp + 1
+        const int ot = 32 * (warp - 18) + lane, kt = ot >> 5, jp = ot & 31;
+        uint4 *xt0 = reinterpret_cast<uint4 *>(sm.xt + (size_t)(kKB * kt + 2 * jp) * NB * 2);
+        for (int i = 0; i < nst && col_major_x<NB>(); i++) {
+            const int s = i % NX;
+            // the previous stage's column-major copy is free, this stage's x tiles have landed
+            if ((i > 0 && !mbar_wait_warp(sm.xtfree, (i - 1) & 1)) || !mbar_wait_warp(&sm.xfull[s], (i / NX) & 1)) {
+                if (lane == 0) report(p.status, kStatusTimeout);
+                break;
+            }
+            {
+                const unsigned char *tile = sm.x + s * XB + kt * NB * 128;
+#pragma unroll
+                for (int q = 0; q < NB / 8; q++) {
+                    uint32_t w[NB];  // rows 8q .. 8q + 7 used
+#pragma unroll
+                    for (int b = 8 * q; b < 8 * q + 8; b++)
+                        w[b] = *reinterpret_cast<const uint32_t *>(tile + sw128_off(b, 2 * jp));
+                    uint4 lo, hi;  // columns 2 jp and 2 jp + 1, rows 8q .. 8q + 7
+                    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(lo.x) : "r"(w[8 * q + 0]), "r"(w[8 * q + 1]));
+                    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(lo.y) : "r"(w[8 * q + 2]), "r"(w[8 * q + 3]));
+                    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(lo.z) : "r"(w[8 * q + 4]), "r"(w[8 * q + 5]));
+                    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(lo.w) : "r"(w[8 * q + 6]), "r"(w[8 * q + 7]));
+                    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(hi.x) : "r"(w[8 * q + 0]), "r"(w[8 * q + 1]));
+                    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(hi.y) : "r"(w[8 * q + 2]), "r"(w[8 * q + 3]));
+                    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(hi.z) : "r"(w[8 * q + 4]), "r"(w[8 * q + 5]));
+                    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(hi.w) : "r"(w[8 * q + 6]), "r"(w[8 * q + 7]));
+                    xt0[q] = lo;
+                    xt0[NB / 8 + q] = hi;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.xempty[s]);  // this warp is done with the ring stage
+                mbar_arrive(sm.xtready);
+            }
+            if (!mbar_wait_warp(sm.xtready, i & 1)) {
+                if (lane == 0) report(p.status, kStatusTimeout);
+                break;
+            }
+            const int c0 = kKB * (kb0 + kKS * i);
+            const int c1 = min(c0 + kKS * kKB, cend);
+            while ((int)(qv[0] & 0xffffu) < c1) {
+                const uint4 *xc = reinterpret_cast<const uint4 *>(sm.xt + (size_t)((int)(qv[0] & 0xffffu) - c0) * NB * 2);
+                const unsigned short vb = (unsigned short)(qv[0] >> 16);
+#pragma unroll
+                for (int q = 0; q < NB / 8; q++) {
+                    const uint4 v = xc[q];
+                    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int t = 0; t < 4; t++)
+                        asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+                            "fma.rn.f32.f16 %0, %3, l, %0;\n\tfma.rn.f32.f16 %1, %3, h, %1;\n\t}"
+                            : "+f"(acc[8 * q + 2 * t]), "+f"(acc[8 * q + 2 * t + 1])
+                            : "r"(vv[t]), "h"(vb));
+                }
+                qv[0] = qv[1];
+                qv[1] = qv[2];
+                qv[2] = qv[3];
+                k++;
+                qv[3] = entry(k + 3);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sm.xtfree);
         }
 #pragma unroll
         for (int b = 0; b < NB; b++) sm.obuf[r * NB + b] = acc[b];
