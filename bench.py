@@ -159,15 +159,40 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ traffic record
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without its // and /* */ comments (string and character
+    literals kept), whitespace-normalised per line."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (" ".join(line.split()) for line in "".join(out).splitlines())
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_source_digest() -> str:
-    """Digest of the library sources; a recorded ncu traffic figure only
-    holds for the sources it was measured on."""
+    """Digest of the library sources without their comments; a recorded ncu
+    traffic figure only holds for the code it was measured on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dense_sparse_quantized_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                h.update(name.encode() + strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

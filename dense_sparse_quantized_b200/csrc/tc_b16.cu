@@ -26,9 +26,12 @@
 //                exact q - zero, one HMUL2 rounds scale*(q - zero) once -- and
 //                stores them into tensor memory (tcgen05.st) as the MMA's A
 //                operand;
-//   warps 18-21  outliers: thread (row) walks its row's CSR entries that fall
-//                in each K-block and accumulates v * x[b][col] in fp32 from the
-//                staged x tile (exact products);
+//   warps 18-21  outliers: the tile's CSR slice is brought into shared memory
+//                by one bulk copy when it fits; thread (row) then walks its
+//                row's entries that fall in each stage and accumulates
+//                v * x[b][col] in fp32 (exact products) from the staged x
+//                tiles -- at 64 activation rows from a column-major copy of
+//                the stage that the four warps write first;
 // after the loop warps 2-5 read the accumulator rows (tcgen05.ld), add the
 // outlier sums, reduce over the cluster and store y.
 //
