@@ -309,10 +309,15 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *sm.tmem_slot;
+    // The next call may start launching; weights, scales and outliers belong
+    // to the handle, so only x (loaded below) and y (stored at the end) wait
+    // for the previous kernel in the stream.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == 0) {
         // x producer: per stage, the kKS x tiles [NB][64] (128-byte swizzle)
         if (lane == 0) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
             int issued = 0;
             for (int i = 0; i < nst; i++) {
                 const int s = i % NX;
@@ -582,6 +587,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
     }
     if (KS > 1) cluster_sync();
     if (epi && rank == 0 && grow < p.rows) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int j = 0; j < KS - 1; j++)
 #pragma unroll
             for (int b = 0; b < NB; b++) part[b] += sm.rbuf[((size_t)j * kTM + r) * NB + b];
@@ -618,19 +624,21 @@ bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_
 
 template <int NB>
 int launch_nb(const TcParams &p, int KS, const CUtensorMap &tx, const CUtensorMap &trec, const CUtensorMap &tzero,
-              __half *y, cudaStream_t st) {
+              __half *y, cudaStream_t st, bool pdl) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(KS, (p.rows + kTM - 1) / kTM, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem_bytes<NB>();
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = KS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, tc_kernel<NB>, tx, trec, tzero, p, KS, y) == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
 }
 
@@ -674,8 +682,11 @@ bool tc_shape_ok(const MatrixView &m) {
 }
 
 // All launches of one product (batch in chunks of 64 rows of x).
+// pdl: programmatic dependent launch (the kernel reads the packed matrix
+// before the previous kernel in the stream has finished) -- only for packed
+// data the handle owns.
 int run_tc(const MatrixView &m, const Split &sp, const int32_t *split_start, int *status, const __half *x,
-           __half *y, int batch, cudaStream_t st) {
+           __half *y, int batch, cudaStream_t st, bool pdl) {
     for (int b0 = 0; b0 < batch; b0 += 64) {
         const int nb = std::min(64, batch - b0);
         const int NB = nb <= 16 ? 16 : nb <= 32 ? 32 : 64;
@@ -706,9 +717,9 @@ int run_tc(const MatrixView &m, const Split &sp, const int32_t *split_start, int
         p.status = status;
         __half *yb = y + (size_t)b0 * m.rows;
         int rc;
-        if (NB == 16) rc = launch_nb<16>(p, sp.KS, tx, trec, tzero, yb, st);
-        else if (NB == 32) rc = launch_nb<32>(p, sp.KS, tx, trec, tzero, yb, st);
-        else rc = launch_nb<64>(p, sp.KS, tx, trec, tzero, yb, st);
+        if (NB == 16) rc = launch_nb<16>(p, sp.KS, tx, trec, tzero, yb, st, pdl);
+        else if (NB == 32) rc = launch_nb<32>(p, sp.KS, tx, trec, tzero, yb, st, pdl);
+        else rc = launch_nb<64>(p, sp.KS, tx, trec, tzero, yb, st, pdl);
         if (rc != DSQ_OK) return rc;
     }
     return DSQ_OK;
@@ -780,7 +791,7 @@ void tc_free(dsq_handle_s *h) {
 int launch_gemv_tc(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t st) {
     if (!tc_covers(h, batch)) return DSQ_ERR_UNSUPPORTED;
     const Split sp = {h->tc.KS, h->tc.nkb, h->tc.kb_per_split};
-    return run_tc(h->view, sp, h->tc.split_start, h->d_status, x, y, batch, st);
+    return run_tc(h->view, sp, h->tc.split_start, h->d_status, x, y, batch, st, true);
 }
 
 }  // namespace dsq
@@ -905,6 +916,8 @@ extern "C" int dsq_gemv_noalloc(const dsq_desc *d, const void *packed_device, si
     noalloc_prep_kernel<<<(unsigned)((n_prep + 255) / 256), 256, 0, st>>>(
         nd.scratch, m.row_ptr, m.csr, m.rows, sp.KS, sp.kb_per_split * kKB);
     if (cudaGetLastError() != cudaSuccess) return DSQ_ERR_CUDA;
+    // no programmatic dependent launch: the packed matrix is the caller's and
+    // the split starts come from the kernel just launched
     return run_tc(m, sp, nd.scratch + kNoAllocStartsOff, (int *)nd.scratch, (const __half *)x, (__half *)y, batch,
-                  st);
+                  st, false);
 }
