@@ -184,15 +184,16 @@ def strip_comments(src: str) -> str:
     return "\n".join(line for line in lines if line)
 
 
-def kernel_source_digest() -> str:
-    """Digest of the library sources without their comments; a recorded ncu
-    traffic figure only holds for the code it was measured on."""
+def kernel_source_digest(files=None) -> str:
+    """Digest of library sources without their comments (all of them, or the
+    named files of the csrc folder); a recorded ncu traffic figure only holds
+    for the code it was measured on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dense_sparse_quantized_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".h")):
-            with open(os.path.join(csrc, name), encoding="utf-8") as f:
-                h.update(name.encode() + strip_comments(f.read()).encode())
+    names = files if files else [n for n in os.listdir(csrc) if n.endswith((".cu", ".h"))]
+    for name in sorted(names):
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -203,7 +204,7 @@ def recorded_traffic(config: str, batch: int):
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)
         e = rec.get(f"{config}_b{batch}")
-        if e and e.get("source_digest") == kernel_source_digest():
+        if e and e.get("source_digest") == kernel_source_digest(e.get("sources")):
             return float(e["dram_bytes_per_launch"]), e.get("note", "")
     except Exception:
         pass
