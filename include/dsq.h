@@ -131,10 +131,16 @@ DSQ_API int dsq_create(const void *packed, size_t bytes, int device, dsq_handle_
  *   y      device fp16 [batch][rows], row-major, 16-byte aligned (may be
  *          NULL only when rows == 0); fully overwritten, each
  *          element written once, rounded to nearest from an fp32 sum.
- *   batch  >= 1.  Batches of 16 and more go through the tensor-core path.
+ *   batch  >= 1.  Affine 3-bit matrices take the tensor-core path from 3
+ *          rows on (from 16 when a row holds more than 256 outliers);
+ *          table matrices take a CUDA-core kernel, 4 rows per launch.
  *   stream cudaStream_t of the handle's device, as void*.
  * x and y are the caller's and must not overlap.  The handle is read-only
  * here, so calls on several streams or threads may run concurrently.
+ * The kernels use programmatic dependent launch: they may start while the
+ * previous kernel in `stream` is still running, but until it has finished
+ * they read only the handle's own device memory; x is read and y written
+ * after it, as with plain stream order.
  * Accuracy: |y - y_exact| <= 1e-3 * sum_j |What[i][j]| * |x[b][j]|.
  * Returns DSQ_OK, DSQ_ERR_INVALID_ARG (NULL or misaligned pointer,
  * batch < 1) or DSQ_ERR_CUDA (launch failure).
