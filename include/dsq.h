@@ -133,7 +133,8 @@ DSQ_API int dsq_create(const void *packed, size_t bytes, int device, dsq_handle_
  *          element written once, rounded to nearest from an fp32 sum.
  *   batch  >= 1.  Affine 3-bit matrices take the tensor-core path from 3
  *          rows on (from 16 when a row holds more than 256 outliers);
- *          table matrices take a CUDA-core kernel, 4 rows per launch.
+ *          table matrices take a CUDA-core kernel, 4 rows per launch;
+ *          affine 4-bit matrices take the one-warp-per-row kernel.
  *   stream cudaStream_t of the handle's device, as void*.
  * x and y are the caller's and must not overlap.  The handle is read-only
  * here, so calls on several streams or threads may run concurrently.
