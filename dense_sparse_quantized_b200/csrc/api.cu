@@ -49,6 +49,7 @@ extern "C" int dsq_create(const void *packed, size_t bytes, int device, dsq_hand
     *out = nullptr;
     BlobHeader hd;
     int rc = parse_blob(packed, bytes, &hd);
+    if (rc == DSQ_OK) rc = check_blob_contents(packed, hd);
     if (rc != DSQ_OK) return rc;
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess) return DSQ_ERR_CUDA;

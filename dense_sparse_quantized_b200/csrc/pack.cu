@@ -78,6 +78,36 @@ int parse_blob(const void *packed, size_t bytes, BlobHeader *out) {
     return DSQ_OK;
 }
 
+// The blob contents the kernels index by: row_ptr (from 0 to nnz, never
+// decreasing) and the CSR columns (below cols, strictly increasing within a
+// row).  Codes, tables, scales and zero points are safe for any bit pattern.
+// Host-side, O(rows + nnz); the blob may sit at any host address.
+int check_blob_contents(const void *packed, const BlobHeader &h) {
+    const uint8_t *b = (const uint8_t *)packed;
+    auto rp = [&](int64_t i) {
+        int32_t v;
+        memcpy(&v, b + h.off_row_ptr + 4 * i, 4);
+        return (int64_t)v;
+    };
+    auto col = [&](int64_t k) {
+        uint32_t v;
+        memcpy(&v, b + h.off_csr + 4 * k, 4);
+        return (int64_t)(v & 0xffffu);
+    };
+    if (rp(0) != 0 || rp(h.rows) != h.nnz) return DSQ_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < h.rows; i++) {
+        const int64_t k0 = rp(i), k1 = rp(i + 1);
+        if (k1 < k0) return DSQ_ERR_INVALID_ARG;
+        int64_t prev = -1;
+        for (int64_t k = k0; k < k1; k++) {
+            const int64_t c = col(k);
+            if (c >= h.cols || c <= prev) return DSQ_ERR_INVALID_ARG;
+            prev = c;
+        }
+    }
+    return DSQ_OK;
+}
+
 }  // namespace dsq
 
 using namespace dsq;

@@ -118,6 +118,10 @@ DSQ_API int dsq_blob_desc(const void *packed, size_t bytes, dsq_desc *out);
  * device allocation it makes (released by dsq_destroy); the blob stays the
  * caller's and may be freed on return.  Synchronous.  The calling thread's
  * current device is left unchanged.
+ * The blob's header and its outlier index (row pointers from 0 to nnz, never
+ * decreasing; columns below cols and increasing within a row) are checked
+ * on the host before any device work; codes, tables and scales are used as
+ * they are.
  * Returns DSQ_OK, DSQ_ERR_INVALID_ARG (NULL out, malformed blob, bad
  * device), DSQ_ERR_UNSUPPORTED (not an sm_100 device), DSQ_ERR_OOM or
  * DSQ_ERR_CUDA.

@@ -255,3 +255,63 @@ def test_three_bit_fields():
         (w0, p0), (w1, p1) = place[c, 0], place[c + 1, 0]
         assert w0 == w1 and p1 == p0 + 16
         assert p0 + 2 <= 9 or (p0 >= 10 and p0 - 10 + 2 <= 9)
+
+
+# --------------------------------------------------------------- blob contents at create
+
+def _create_rc(blob: bytes) -> int:
+    """dsq_create's status for a blob; a handle made on a GPU machine is freed.
+    Without a device a blob that passes validation ends in DSQ_ERR_CUDA."""
+    lib = dsq.library()
+    h = ctypes.c_void_p()
+    rc = lib.dsq_create(blob, len(blob), 0, ctypes.byref(h))
+    if rc == dsq.DSQ_OK:
+        lib.dsq_destroy(h)
+    return rc
+
+
+def _offsets(blob: bytes):
+    rows = int(np.frombuffer(blob[16:20], np.int32)[0])
+    off_rp, off_csr = (int(v) for v in np.frombuffer(blob[64:80], np.uint64))
+    return rows, off_rp, off_csr
+
+
+@pytest.mark.parametrize("bits,mode", [(3, "lut"), (4, "lut"), (3, "affine"), (4, "affine")])
+def test_create_accepts_packed_blobs(bits, mode):
+    for rows, cols, dens in ((7, 48, 0.05), (33, 1024, 0.02), (5, 16, 0.0), (1, 4096, 0.01)):
+        p = synth.make_problem(rows, cols, bits, mode, dens, "uniform" if dens else "none", 9, 1)
+        assert _create_rc(dsq.pack_problem(p)) in (dsq.DSQ_OK, dsq.DSQ_ERR_CUDA), (rows, cols, dens)
+
+
+def test_create_rejects_corrupted_csr():
+    """A blob whose row pointers or CSR columns would send a kernel outside
+    its buffers is refused before any device work."""
+    p = synth.make_problem(6, 64, 3, "affine", 0.1, "uniform", 4, 1)
+    blob = dsq.pack_problem(p)
+    assert _create_rc(blob) in (dsq.DSQ_OK, dsq.DSQ_ERR_CUDA)
+    rows, off_rp, off_csr = _offsets(blob)
+    rp = np.frombuffer(blob[off_rp:off_rp + 4 * (rows + 1)], np.int32).copy()
+    busy = int(np.argmax(np.diff(rp)))  # a row with at least two entries
+    assert rp[busy + 1] - rp[busy] >= 2
+
+    def with_rp(new_rp):
+        b = bytearray(blob)
+        b[off_rp:off_rp + 4 * (rows + 1)] = np.asarray(new_rp, np.int32).tobytes()
+        return bytes(b)
+
+    def with_entry(k, col):
+        b = bytearray(blob)
+        e = int(np.frombuffer(blob[off_csr + 4 * k:off_csr + 4 * k + 4], np.uint32)[0])
+        b[off_csr + 4 * k:off_csr + 4 * k + 4] = np.uint32((e & 0xFFFF0000) | col).tobytes()
+        return bytes(b)
+
+    bad = rp.copy(); bad[0] = 1
+    assert _create_rc(with_rp(bad)) == dsq.DSQ_ERR_INVALID_ARG          # does not start at 0
+    bad = rp.copy(); bad[-1] -= 1
+    assert _create_rc(with_rp(bad)) == dsq.DSQ_ERR_INVALID_ARG          # does not end at nnz
+    bad = rp.copy(); bad[busy + 1] = bad[busy] - 1 if bad[busy] > 0 else -1
+    assert _create_rc(with_rp(bad)) == dsq.DSQ_ERR_INVALID_ARG          # decreasing
+    k = int(rp[busy])
+    assert _create_rc(with_entry(k, p.cols)) == dsq.DSQ_ERR_INVALID_ARG  # column out of range
+    c_next = int(np.frombuffer(blob[off_csr + 4 * (k + 1):off_csr + 4 * (k + 2)], np.uint32)[0]) & 0xFFFF
+    assert _create_rc(with_entry(k, c_next)) == dsq.DSQ_ERR_INVALID_ARG  # repeated column in a row
