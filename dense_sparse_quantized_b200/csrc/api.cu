@@ -9,6 +9,10 @@
 
 using namespace dsq;
 
+namespace dsq {
+int check_blob_contents(const void *packed, const BlobHeader &h);  // pack.cu
+}
+
 namespace {
 
 // Makes `device` current for the scope and restores the caller's device.

@@ -15,7 +15,6 @@ double half_bits_to_double(uint16_t h);
 int check_desc(const dsq_desc *d);
 void plan_blob(const dsq_desc *d, BlobHeader *h);
 int parse_blob(const void *packed, size_t bytes, BlobHeader *out);
-int check_blob_contents(const void *packed, const BlobHeader &h);
 
 // Device view of one packed matrix (pointers into the handle's device copy
 // of the blob).
