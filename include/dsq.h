@@ -208,7 +208,9 @@ DSQ_API int dsq_destroy(dsq_handle_t h);
  * d             host; the blob's shape (as dsq_blob_desc reports it).
  * packed_device device; the dsq_pack blob copied verbatim, `bytes` long
  *               (exactly the size dsq_pack reported), 256-byte aligned.
- *               Read only; the caller owns it.
+ *               Read only; the caller owns it.  Being on the device, its
+ *               contents are not checked as dsq_create checks them: pass
+ *               only blobs that dsq_pack wrote.
  * x, y, batch, stream  as for dsq_gemv (fp16 [batch][cols] / [batch][rows],
  *               16-byte aligned, on the current device).
  *
