@@ -265,3 +265,32 @@ def test_streams_and_repeat_calls_agree():
     s.synchronize()
     torch.cuda.synchronize()
     assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+
+
+@pytest.mark.parametrize("mode,batch", [("affine", 1), ("affine", 16), ("lut", 1), ("lut", 4)])
+def test_back_to_back_calls_read_the_x_just_written(mode, batch):
+    """The kernels start before the previous kernel in the stream ends
+    (programmatic dependent launch) and must still read the x that kernel
+    wrote and write y after it: x is rewritten by a copy kernel right before
+    every call, with no synchronisation, and each y must equal, bit for bit,
+    the y of the same x computed in isolation."""
+    p = synth.make_problem(1024, 2048, 3, mode, 0.01, "uniform", 31, batch)
+    rng = np.random.default_rng(5)
+    xs = [to_dev(synth.f16_bits(rng.standard_normal((batch, p.cols)))) for _ in range(6)]
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        ref = []
+        for xv in xs:
+            ref.append(h.gemv(xv).clone())
+            torch.cuda.synchronize()
+        x = torch.empty_like(xs[0])
+        y = torch.empty((batch, p.rows), dtype=torch.float16, device="cuda")
+        got = []
+        for _ in range(3):
+            for xv in xs:
+                x.copy_(xv)        # a kernel writes x ...
+                h.gemv(x, y)       # ... and the product reads it at once
+                got.append(y.clone())
+        torch.cuda.synchronize()
+        h.check()
+    for i, g in enumerate(got):
+        assert torch.equal(g.view(torch.int16), ref[i % len(xs)].view(torch.int16)), i
