@@ -37,7 +37,7 @@ extern "C" const char *dsq_status_string(int status) {
     switch (status) {
         case DSQ_OK: return "DSQ_OK";
         case DSQ_ERR_INVALID_ARG: return "DSQ_ERR_INVALID_ARG: invalid argument";
-        case DSQ_ERR_UNSUPPORTED: return "DSQ_ERR_UNSUPPORTED: not supported by this build";
+        case DSQ_ERR_UNSUPPORTED: return "DSQ_ERR_UNSUPPORTED: outside what the library supports";
         case DSQ_ERR_CUDA: return "DSQ_ERR_CUDA: CUDA runtime or launch failure";
         case DSQ_ERR_OOM: return "DSQ_ERR_OOM: device allocation failed";
         case DSQ_ERR_BUFFER_TOO_SMALL: return "DSQ_ERR_BUFFER_TOO_SMALL: output buffer too small";

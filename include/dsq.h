@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
     DSQ_OK = 0,
     DSQ_ERR_INVALID_ARG = -1,     /* a NULL pointer, a size or value out of range, a malformed blob */
-    DSQ_ERR_UNSUPPORTED = -2,     /* well-formed but outside this build (e.g. cols > 65535) */
+    DSQ_ERR_UNSUPPORTED = -2,     /* well-formed but outside what the library supports (e.g. cols > 65535) */
     DSQ_ERR_CUDA = -3,            /* a CUDA runtime call or a kernel launch failed */
     DSQ_ERR_OOM = -4,             /* device allocation failed */
     DSQ_ERR_BUFFER_TOO_SMALL = -5,/* output buffer smaller than required; size reported */

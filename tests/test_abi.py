@@ -260,7 +260,7 @@ def test_three_bit_fields():
 # --------------------------------------------------------------- blob contents at create
 
 def _create_rc(blob: bytes) -> int:
-    """dsq_create's status for a blob; a handle made on a GPU machine is freed.
+    """dsq_create's status for a blob; a handle made where a GPU is present is freed.
     Without a device a blob that passes validation ends in DSQ_ERR_CUDA."""
     lib = dsq.library()
     h = ctypes.c_void_p()
