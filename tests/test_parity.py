@@ -172,7 +172,7 @@ def test_all_outlier_rows(orc, mode):
         check_y(gemv(h, q.x, 2), y_ref, bound, "all-outlier rows")
 
 
-@pytest.mark.parametrize("batch", [16, 40])
+@pytest.mark.parametrize("batch", [16, 32, 40])
 def test_tile_outliers_staged_and_not(orc, batch):
     """Tensor-core path: the first 128-row tile holds 300 outliers per row, more
     than the CSR slice kept in shared memory, so its outlier warps read the
