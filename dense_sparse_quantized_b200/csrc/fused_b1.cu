@@ -15,17 +15,18 @@
 // one thread per row adds the column partials and the row's piece sums, in a
 // fixed order, and stores y.
 //
-// Affine decode.  A pair of 3-bit codes sits at the same bit (0, 3 or 6) of
-// both 16-bit halves of a word, or of the word shifted right by 10, so one
-// AND yields two fp16 subnormals q * 2^(k-24), exact.  A mixed-precision FMA
-// (fp32 += fp16 * fp16: the product of two fp16 is exact in fp32) adds
-// q * x * 2^(k-24) into one of three fp32 sums per group, by k; per group g
-// of 16 columns
-//     t_g = sum_c q_c x_c - zero_g * X_g        (X_g = sum of the group's x)
-//     acc += scale_g * t_g
-// i.e. scale*(q - zero) factored out of the group sum; 2^-24 is removed once
-// per row.  x stays in its fp16 form in registers: nothing is rounded but
-// the fp32 sums.
+// Affine decode.  A pair of 3-bit codes sits at the same bit h (0, 3 or 6)
+// of both 16-bit halves of a word, or of the word shifted right by 10.  One
+// LOP3 keeps the pair and ORs in the exponent of M_h = 2^(10-h): each half is
+// then the fp16 number M_h + q (the code lands in the mantissa in units of
+// 1).  One HSUB2 of M_h + zero (exact: both operands lie within a factor of
+// two) leaves q - zero, a small integer, and two mixed-precision FMAs (fp32
+// += fp16 * fp16, whose product is exact in fp32) add (q - zero) * x to the
+// group's fp32 sum; the fp16 scale multiplies each group sum once.  The zero
+// point is taken off every code before its product, so the rounding error of
+// a group sum follows sum |q - zero| |x|, the weights' own share of the
+// error bound, whatever the range of x.  x stays in its fp16 form in
+// registers: nothing is rounded but the fp32 sums.
 //
 // Table decode.  Every lane of a 2^b-lane segment holds one centroid of the
 // current row (fp32); shfl.idx over that segment reads only the low b bits of
@@ -44,7 +45,8 @@ namespace {
 constexpr int kMaxWarps = 24;  // warps per CTA
 constexpr int kThreads = kMaxWarps * 32;
 constexpr int kDepth = 4;      // table kernel: rows each lane has in flight (cp.async ring stages), a power of 2
-constexpr int kD = 6;          // affine kernel: rows each lane has in flight (cp.async ring stages)
+constexpr int kD = 8;          // affine kernel: rows each lane has in flight (cp.async ring stages)
+constexpr int kRB = 4;         // affine kernel: rows decoded per step, reduced together (divides kD)
 constexpr int kHeavyPieces = 32;  // rows with more pieces are summed by a whole warp
 constexpr int kPre = 4;          // affine kernel: ring stages requested before the dependency wait
 // shared-memory header: mbarriers of the staged CSR + piece lists and of the
@@ -109,6 +111,37 @@ __device__ __forceinline__ float warp_sum(float r) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(kFull, r, o);
     return r;
+}
+
+// v[0..NB-1] (one value per activation row) summed over the warp in one
+// transposed butterfly; afterwards lane l holds the total of activation row
+// bn_row<NB>(l), in a fixed order.
+template <int NB>
+__device__ __forceinline__ float reduce_rows(float (&v)[NB], int lane) {
+    int o = 16;
+#pragma unroll
+    for (int n = NB; n > 1; n >>= 1, o >>= 1) {
+        const bool hi = lane & o;
+#pragma unroll
+        for (int i = 0; i < n / 2; i++) {
+            const float send = hi ? v[i] : v[i + n / 2], keep = hi ? v[i + n / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+    }
+#pragma unroll
+    for (; o >= 1; o >>= 1) v[0] += __shfl_xor_sync(kFull, v[0], o);
+    return v[0];
+}
+// The row whose total reduce_rows leaves in lane l: the halvings at lane
+// bits 4, 3, 2 pick it, high bit first; lanes with the remaining low bits
+// zero store it.
+template <int NB>
+__device__ __forceinline__ int bn_row(int lane) {
+    return NB == 8 ? (lane >> 2) & 7 : NB == 4 ? (lane >> 3) & 3 : NB == 2 ? (lane >> 4) & 1 : 0;
+}
+template <int NB>
+__device__ __forceinline__ bool bn_store_lane(int lane) {
+    return (lane & (NB == 8 ? 3 : NB == 4 ? 7 : NB == 2 ? 15 : 31)) == 0;
 }
 
 // Thread t sums pieces t, t + blockDim, ... of the tile (each <= kPieceMax
@@ -190,42 +223,51 @@ __device__ __forceinline__ void mfma_pair(float &lo, float &hi, uint32_t p, uint
         : "r"(p), "r"(xh));
 }
 
-// fp32 value of a small unsigned integer n < 2^23 (exact).
-__device__ __forceinline__ float small_u2f(uint32_t n) { return __uint_as_float(n | 0x4B000000u) - 8388608.f; }
+// fp16 exponent pattern of M_h = 2^(10-h) in both halves, for a code field
+// at bit h = 3k of each half (1024, 128, 16).
+__host__ __device__ constexpr uint32_t magic_of(int k) {
+    return k == 0 ? 0x64006400u : k == 1 ? 0x58005800u : 0x4C004C00u;
+}
 
-// Affine 3-bit slot record v (3 code words + scale pair), zero byte zb, the
-// lane's 32 columns of x as fp16 pairs xh[m] = (x[2m], x[2m+1]) and the
-// group sums of x times 2^-24: returns
-// scale_A*(sum_A q x - zA X_A) + scale_B*(...), in units of 2^-24.
-__device__ __forceinline__ float decode_aff3(const uint4 v, uint32_t zb, const uint32_t (&xh)[16], float XAt,
-                                             float XBt) {
+// (a & mask) | c in one LOP3.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t c) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(c));
+    return r;
+}
+
+// Both halves of a - b in fp16 (used where the difference is exact).
+__device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Affine 3-bit slot record v (3 code words + scale pair), zero byte zb and
+// the lane's 32 columns of x as fp16 pairs xh[m] = (x[2m], x[2m+1]):
+// returns scale_A * sum_A (q - zA) x + scale_B * sum_B (q - zB) x.
+__device__ __forceinline__ float decode_aff3(const uint4 v, uint32_t zb, const uint32_t (&xh)[16]) {
     const uint32_t w[3] = {v.x, v.y, v.z};
     const uint32_t sh[3] = {v.x >> 10, v.y >> 10, v.z >> 10};
-    float acc[2][3][2];  // [group][k / 3][low, high half]
+    const uint32_t z[2] = {zb & 15u, (zb >> 4) & 15u};
+    uint32_t mz[2][3];  // M_h + zero in both halves, per group and field class
 #pragma unroll
     for (int g = 0; g < 2; g++)
 #pragma unroll
-        for (int k = 0; k < 3; k++) acc[g][k][0] = acc[g][k][1] = 0.f;
+        for (int k = 0; k < 3; k++) mz[g][k] = z[g] * (0x00010001u << (3 * k)) + magic_of(k);
+    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // [group][low, high half]
 #pragma unroll
     for (int m = 0; m < 15; m++) {  // pair m = columns 2m, 2m+1: word m/5, slot j = m%5
-        const int i = m / 5, j = m % 5, k = j < 3 ? j : j - 3;
-        const uint32_t pr = (j < 3 ? w[i] : sh[i]) & (0x00070007u << (3 * k));
-        const int g = m < 8 ? 0 : 1;
-        mfma_pair(acc[g][k][0], acc[g][k][1], pr, xh[m]);
+        const int i = m / 5, j = m % 5, k = j < 3 ? j : j - 3, g = m < 8 ? 0 : 1;
+        const uint32_t pr = and_or(j < 3 ? w[i] : sh[i], 0x00070007u << (3 * k), magic_of(k));
+        mfma_pair(acc[g][0], acc[g][1], hsub2_bits(pr, mz[g][k]), xh[m]);
     }
     // columns 30 (low half) and 31 (high half): bit k is bit 9 / 25 of word k
     const uint32_t t15 = ((w[0] >> 9) & 0x00010001u) | ((w[1] >> 8) & 0x00020002u) | ((w[2] >> 7) & 0x00040004u);
-    mfma_pair(acc[1][0][0], acc[1][0][1], t15, xh[15]);
-    float t[2];
-#pragma unroll
-    for (int g = 0; g < 2; g++)
-        t[g] = fmaf(acc[g][2][0] + acc[g][2][1], 0x1p-6f,
-                    fmaf(acc[g][1][0] + acc[g][1][1], 0x1p-3f, acc[g][0][0] + acc[g][0][1]));
+    mfma_pair(acc[1][0], acc[1][1], hsub2_bits(t15 | magic_of(0), mz[1][0]), xh[15]);
     const float sA = __half2float(__ushort_as_half((unsigned short)(v.w & 0xffffu)));
     const float sB = __half2float(__ushort_as_half((unsigned short)(v.w >> 16)));
-    const float zA = small_u2f(zb & 15u), zB = small_u2f((zb >> 4) & 15u);
-    const float r = sA * fmaf(-zA, XAt, t[0]);
-    return fmaf(sB, fmaf(-zB, XBt, t[1]), r);
+    return fmaf(sB, acc[1][0] + acc[1][1], sA * (acc[0][0] + acc[0][1]));
 }
 
 // Table slot: code words w[0..BITS-1], this row's centroid held by the lane.
@@ -346,11 +388,14 @@ __device__ __forceinline__ void read_row(uint32_t rs, uint32_t rb, uint4 &v, uin
 // lanes 0, 1 the group's zero bytes, kD rows ahead, into the warp's ring
 // (cp.async, one commit group per row); each lane reads back its record and
 // zero byte.  A lane's wait covers only its own copies, so a warp barrier
-// follows each wait before the zero bytes are read; the refill of a stage
-// comes after the row's warp reduction, when every lane has read it.
+// follows each wait before the zero bytes are read.  Rows go kRB at a time:
+// each lane decodes its slot of kRB rows, one transposed butterfly sums the
+// kRB partials over the warp (4 rows: 7 shuffles instead of 20), and the
+// stages are refilled after it, when every lane has read them.
 template <int NT, int PER_SM>
 __global__ void __launch_bounds__(NT, PER_SM)
 b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
+    static_assert(kD % kRB == 0, "ring depth");
     extern __shared__ __align__(128) unsigned char smem[];
     const MatrixView &m = p.m;
     const int S = m.slots, C = p.C, R = p.R;
@@ -389,51 +434,64 @@ b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y)
             copy_row<d * kAffStageB>(rs, rz, lb, d < nj, zl);
             lb += step;
         });
-        float XA = 0.f, XB = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; i++) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&xh[i]));
-            if (i < 8) XA += f.x + f.y;
-            else XB += f.x + f.y;
-        }
-        const float XAt = XA * 0x1p-24f, XBt = XB * 0x1p-24f;
         if (rg == 0) stage_x(smem, p, s, xh);
 
-        uint32_t part = smem_u32(smem + p.off_part) + 4 * (rg * C + cw);
+        // partial of this warp's row jj at part + jj * pstep
+        const uint32_t part = smem_u32(smem + p.off_part) + 4 * (rg * C + cw);
         const uint32_t pstep = 4 * R * C;
+        const int my_row = bn_row<kRB>(lane);
+        const bool stores = bn_store_lane<kRB>(lane);
         int j = 0;
         for (; j + kD <= nj; j += kD) {
-            unroll<0, kD>([&](auto dc) {
-                constexpr int d = decltype(dc)::value;
-                cp_async_wait<kD - 1>();  // this lane's copies of row j + d have landed ...
-                __syncwarp();             // ... and every lane's (lanes 0, 1 copy the zero bytes)
-                uint4 v;
-                uint32_t zb;
-                read_row<d * kAffStageB>(rs, rb, v, zb);
-                const float r = warp_sum(decode_aff3(v, zb, xh, XAt, XBt));
-                // every lane holds the sum; the stores coincide
-                asm volatile("st.shared.f32 [%0], %1;" ::"r"(part), "f"(r) : "memory");
-                part += pstep;
-                // refill the stage just read with row j + d + kD
-                copy_row<d * kAffStageB>(rs, rz, lb, j + d + kD < nj, zl);
-                lb += step;
+            unroll<0, kD / kRB>([&](auto ec) {
+                constexpr int e = decltype(ec)::value;
+                cp_async_wait<kD - kRB>();  // this lane's copies of rows j + kRB e .. have landed ...
+                __syncwarp();               // ... and every lane's (lanes 0, 1 copy the zero bytes)
+                float v[kRB];
+                unroll<0, kRB>([&](auto rc) {
+                    constexpr int d = kRB * e + decltype(rc)::value;
+                    uint4 rec;
+                    uint32_t zb;
+                    read_row<d * kAffStageB>(rs, rb, rec, zb);
+                    v[decltype(rc)::value] = decode_aff3(rec, zb, xh);
+                });
+                const float t = reduce_rows<kRB>(v, lane);
+                if (stores)
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(part + (j + kRB * e + my_row) * pstep), "f"(t)
+                                 : "memory");
+                // every lane has read the stages before they are refilled: lane 0's
+                // shuffles above waited for every lane's, which consumed its loads
+                unroll<0, kRB>([&](auto rc) {
+                    constexpr int d = kRB * e + decltype(rc)::value;
+                    copy_row<d * kAffStageB>(rs, rz, lb, j + d + kD < nj, zl);
+                    lb += step;
+                });
             });
         }
         cp_async_wait<0>();
         __syncwarp();
-        for (int d = 0; j < nj; j++, d++) {
-            uint4 v;
-            uint32_t zb;
-            read_row<0>(rs + d * kAffStageB, rb + d * kAffStageB, v, zb);
-            const float r = warp_sum(decode_aff3(v, zb, xh, XAt, XBt));
-            asm volatile("st.shared.f32 [%0], %1;" ::"r"(part), "f"(r) : "memory");
-            part += pstep;
+        // the last nj - j < kD rows, all landed: kRB at a time, missing rows as 0
+        for (int d0 = 0; j + d0 < nj; d0 += kRB) {
+            float v[kRB];
+#pragma unroll
+            for (int r = 0; r < kRB; r++) {
+                v[r] = 0.f;
+                if (j + d0 + r < nj) {
+                    uint4 rec;
+                    uint32_t zb;
+                    read_row<0>(rs + (d0 + r) * kAffStageB, rb + (d0 + r) * kAffStageB, rec, zb);
+                    v[r] = decode_aff3(rec, zb, xh);
+                }
+            }
+            const float t = reduce_rows<kRB>(v, lane);
+            if (stores && j + d0 + my_row < nj)
+                asm volatile("st.shared.f32 [%0], %1;" ::"r"(part + (j + d0 + my_row) * pstep), "f"(t) : "memory");
         }
     }
     // the outliers, from the staged CSR entries and x
     if (wait_stage(smem, kBarX, p) && wait_stage(smem, kBarCsr, p)) reduce_pieces(td, smem, p);
     __syncthreads();
-    finalize(td, smem, p, 0x1p24f, y);
+    finalize(td, smem, p, 1.0f, y);
 }
 
 template <int KIND>  // 3: LUT 3-bit, 4: LUT 4-bit
@@ -537,37 +595,6 @@ b1_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) 
 
 constexpr int kMaxWarpsN = 12;  // batched table kernel: fewer warps, room for x of 4 rows in registers
 constexpr int kThreadsN = kMaxWarpsN * 32;
-
-// v[0..NB-1] (one value per activation row) summed over the warp in one
-// transposed butterfly; afterwards lane l holds the total of activation row
-// bn_row<NB>(l), in a fixed order.
-template <int NB>
-__device__ __forceinline__ float reduce_rows(float (&v)[NB], int lane) {
-    int o = 16;
-#pragma unroll
-    for (int n = NB; n > 1; n >>= 1, o >>= 1) {
-        const bool hi = lane & o;
-#pragma unroll
-        for (int i = 0; i < n / 2; i++) {
-            const float send = hi ? v[i] : v[i + n / 2], keep = hi ? v[i + n / 2] : v[i];
-            v[i] = keep + __shfl_xor_sync(kFull, send, o);
-        }
-    }
-#pragma unroll
-    for (; o >= 1; o >>= 1) v[0] += __shfl_xor_sync(kFull, v[0], o);
-    return v[0];
-}
-// The row whose total reduce_rows leaves in lane l: the halvings at lane
-// bits 4, 3, 2 pick it, high bit first; lanes with the remaining low bits
-// zero store it.
-template <int NB>
-__device__ __forceinline__ int bn_row(int lane) {
-    return NB == 8 ? (lane >> 2) & 7 : NB == 4 ? (lane >> 3) & 3 : (lane >> 4) & 1;
-}
-template <int NB>
-__device__ __forceinline__ bool bn_store_lane(int lane) {
-    return (lane & (NB == 8 ? 3 : NB == 4 ? 7 : 15)) == 0;
-}
 
 // Table rows, NB activation rows at once (NB = 2 or 4; nb <= NB real).
 // As the batch-1 table kernel, but each lane keeps its 32 columns of x for

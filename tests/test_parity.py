@@ -294,3 +294,70 @@ def test_back_to_back_calls_read_the_x_just_written(mode, batch):
         h.check()
     for i, g in enumerate(got):
         assert torch.equal(g.view(torch.int16), ref[i % len(xs)].view(torch.int16)), i
+
+
+# ------------------------------------------------------------- wide-range activations
+
+F16_OVERFLOW = 65520.0   # |v| at or above this rounds to inf in fp16
+
+
+def zero_columns(p, cols):
+    """p with What[:, cols] == 0 exactly: every code there set to its group's
+    zero point (the dense weight decodes to 0, as at a hole) and the outliers
+    on those columns dropped."""
+    codes = p.codes.copy()
+    z = p.zeros.view(np.float16).astype(np.uint8)
+    codes[:, cols] = z[:, cols // synth.GROUP]
+    keep = ~np.isin(p.col_idx, cols)
+    rows = np.repeat(np.arange(p.rows), np.diff(p.row_ptr))[keep]
+    rp = np.concatenate([[0], np.cumsum(np.bincount(rows, minlength=p.rows))]).astype(np.int32)
+    return edited(p, codes=codes, row_ptr=rp, col_idx=p.col_idx[keep].astype(np.int32),
+                  values=p.values[keep])
+
+
+def wide_problem(p, batch, per_group, seed, big=60000.0, small=1e-4):
+    """The matrix with exact zeros on a few columns, and activations spanning
+    the fp16 range: +-`big` on those columns, |x| ~ `small` everywhere else.
+    The large entries add nothing to y or to the error bound, so a kernel
+    whose rounding error follows them (a zero point subtracted after the
+    group sum, say) shows it.  per_group False: 3 columns; True: one column
+    in every group of 16."""
+    rng = np.random.default_rng(seed)
+    if per_group:
+        cols = np.arange(0, p.cols, synth.GROUP) + rng.integers(0, synth.GROUP, p.cols // synth.GROUP)
+    else:
+        cols = np.sort(rng.choice(p.cols, 3, replace=False))
+    q = zero_columns(p, cols)
+    x = small * (1.0 + rng.random((batch, p.cols))) * rng.choice([-1.0, 1.0], (batch, p.cols))
+    x[:, cols] = big * rng.choice([-1.0, 1.0], (batch, cols.size))
+    return q, synth.f16_bits(x)
+
+
+@pytest.mark.parametrize("per_group", [False, True])
+@pytest.mark.parametrize("batch", [1, 2, 3, 16])
+def test_wide_range_x_c2(orc, per_group, batch):
+    """c2 (11008 x 4096, 3-bit affine) with activations near +-6e4 on columns
+    where every weight is exactly 0 and ~1e-4 elsewhere, through every path
+    an affine 3-bit matrix takes (batch-1 kernel, once per row at batch 2,
+    tensor cores from batch 3 / 16); every row against the oracle."""
+    p, _ = config("c2")
+    q, xb = wide_problem(p, batch, per_group, 40 + batch)
+    with dsq.Handle(dsq.pack_problem(q)) as h:
+        y = gemv(h, xb, batch)
+    y_ref, bound = orc.gemv(q, x=xb)
+    check_y(y, y_ref, bound, f"c2 wide-range x per_group={per_group} B={batch}")
+
+
+@pytest.mark.parametrize("rows,cols", [(256, 1024), (130, 4096), (64, 24640)])
+@pytest.mark.parametrize("per_group", [False, True])
+@pytest.mark.parametrize("batch", [1, 4, 16])
+def test_wide_range_x_small_affine(orc, rows, cols, per_group, batch):
+    """Small affine 3-bit shapes with the same activations; 24640 columns
+    exceed the batch-1 kernel's 24 column groups and run the generic
+    kernel."""
+    p = synth.make_problem(rows, cols, 3, "affine", 0.01, "uniform", rows + cols, 1)
+    q, xb = wide_problem(p, batch, per_group, 7 * batch + rows)
+    with dsq.Handle(dsq.pack_problem(q)) as h:
+        y = gemv(h, xb, batch)
+    y_ref, bound = orc.gemv(q, x=xb)
+    check_y(y, y_ref, bound, f"{rows}x{cols} wide-range per_group={per_group} B={batch}")
