@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = ("dense+sparse 3-bit GEMV µs/call and GB/s as fraction of HBM peak (1×B200)")
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal (~8 TB/s)
 
 
 def parse_args(argv=None):
@@ -213,28 +214,63 @@ def recorded_traffic(config: str, batch: int):
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_rate(p, seconds: float, rows=None):
+def cpu_info():
+    """(logical CPUs usable by this process, CPU model string)."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except Exception:
+        pass
+    return n, model
+
+
+def oracle_rate(p, seconds: float, rows=None, threads: int = 1, x=None):
     """Time the oracle (decode + CSR + fp64 product) on host cores: repeated
-    calls until `seconds` elapse.  Returns (GB/s on canonical bytes of the
-    rows covered, calls, seconds)."""
+    calls over `rows` (all rows by default) until `seconds` elapse.  With
+    threads > 1 the rows are cut into `threads` contiguous slices that the
+    unmodified single-threaded oracle computes concurrently (its C entry
+    point releases the GIL).  Returns (GB/s on canonical bytes of the rows
+    covered, calls, seconds)."""
     import oracle
+    from concurrent.futures import ThreadPoolExecutor
     orc = oracle.load()
-    frac = 1.0 if rows is None else len(rows) / p.rows
+    rows = np.arange(p.rows, dtype=np.int32) if rows is None else np.asarray(rows, dtype=np.int32)
+    frac = len(rows) / p.rows
     bytes_call = p.canonical_bytes(p.batch) * frac
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        orc.gemv(p, rows=rows)
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
+    slices = [s for s in np.array_split(rows, max(1, threads)) if s.size]
+    xv = p.x[:p.batch] if x is None else x
+    with ThreadPoolExecutor(max_workers=len(slices)) as pool:
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            list(pool.map(lambda r: orc.gemv(p, x=xv, rows=r), slices))
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
     return bytes_call * n / el / 1e9, n, el
+
+
+def gpu_config(args, p, canon):
+    """The workload keys both arms report."""
+    import synth
+    return {"workload": f"{args.config}: {synth.describe(args.config)}", "batch": args.batch,
+            "rows": p.rows, "cols": p.cols, "bits": p.bits, "mode": p.mode, "nnz": p.nnz,
+            "canonical_bytes_per_call": canon}
 
 
 def run_reference(args):
     """The oracle, as it stands, on the host: one step = the oracle over a
-    fixed row sample of the workload."""
+    fixed row sample of the workload, computed by the unmodified
+    single-threaded oracle on every host core (row slices in threads)."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
@@ -242,28 +278,35 @@ def run_reference(args):
     import synth
     p = synth.make_config(args.config, batch=args.batch)
     orc = oracle.load()
+    ncpu, model = cpu_info()
     rows = np.arange(0, p.rows, 16, dtype=np.int32)
     frac = len(rows) / p.rows
-    bytes_step = p.canonical_bytes(p.batch) * frac
-    for _ in range(args.warmup):
-        orc.gemv(p, rows=rows)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        orc.gemv(p, rows=rows)
-    el = time.perf_counter() - t0
+    canon = p.canonical_bytes(args.batch)
+    bytes_step = canon * frac
+    slices = [r for r in np.array_split(rows, ncpu) if r.size]
+    from concurrent.futures import ThreadPoolExecutor
+    xv = p.x[:args.batch]
+    with ThreadPoolExecutor(max_workers=len(slices)) as pool:
+        step = lambda: list(pool.map(lambda r: orc.gemv(p, x=xv, rows=r), slices))  # noqa: E731
+        for _ in range(args.warmup):
+            step()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            step()
+        el = time.perf_counter() - t0
     ms = el / args.steps * 1e3
     gbs = bytes_step / (el / args.steps) / 1e9
     sample = (f"every 16th output row ({len(rows)} of {p.rows}) of {args.config} per step, "
-              f"batch {p.batch}; bytes scaled to those rows")
+              f"batch {p.batch}; bytes scaled to those rows; the single-threaded oracle on "
+              f"{len(slices)} row slices in parallel threads")
     line = {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "us_per_call_full_layer": ms * 1e3 / frac, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": f"{args.config}: {synth.describe(args.config)}",
-                       "batch": args.batch},
-            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "config": gpu_config(args, p, canon),
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": len(slices), "kind": "oracle",
+                             "sample": sample, "nproc": ncpu, "cpu_model": model},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -308,9 +351,10 @@ def run_dsq(args):
             call(i)
     stream.synchronize()
 
-    # capture the K timed calls as graphs of G calls (G a multiple of copies)
+    # capture the K timed calls as graphs of G calls (G a multiple of copies,
+    # about 120 calls, so the replays also give a per-call distribution)
     K = args.steps
-    G = min(K, max(copies, (1000 // copies) * copies))
+    G = min(K, copies * max(1, 120 // copies))
     graphs = []
     with torch.cuda.stream(stream):
         for start in range(0, K, G):
@@ -328,17 +372,41 @@ def run_dsq(args):
 
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in graphs]
     barrier(dist, device)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks, torch.cuda.stream(stream):
         ev0.record(stream)
-        for g in graphs:
+        for g, mk in zip(graphs, marks):
             g.replay()
+            mk.record(stream)
         ev1.record(stream)
         ev1.synchronize()
     torch.cuda.synchronize()
     barrier(dist, device)
     t_ms = ev0.elapsed_time(ev1)
+    # per-call time of each replay (calls of one graph, back to back)
+    sizes = [min(G, K - s0) for s0 in range(0, K, G)]
+    per_replay, prev = [], ev0
+    for mk, n in zip(marks, sizes):
+        per_replay.append(prev.elapsed_time(mk) * 1e3 / n)
+        prev = mk
+
+    # latency of one isolated call on the device: a short device-side sleep
+    # holds the stream while the host enqueues the events and the call, so
+    # the call neither overlaps a neighbouring call nor waits for the host
+    iso = []
+    with torch.cuda.stream(stream):
+        for i in range(60):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            stream.synchronize()
+            torch.cuda._sleep(200000)   # ~0.1 ms of device time
+            a.record(stream)
+            call(i)
+            b.record(stream)
+            b.synchronize()
+            if i >= 10:
+                iso.append(a.elapsed_time(b) * 1e3)
     for h in handles:
         h.check()     # raises if a kernel gave up a bounded wait
     t_max, units = reduce_max_sum(dist, t_ms, canon * K, device)
@@ -372,13 +440,22 @@ def run_dsq(args):
     e2e_max, e2e_units = reduce_max_sum(dist, e2e_ms, canon * e2e_steps, device)
     e2e_value = e2e_units / (e2e_max * 1e-3) / 1e9
 
-    # ---- CPU baseline: the oracle as it stands, rank 0, N = 1 only
+    # ---- CPU baseline: the oracle as it stands, rank 0, N = 1 only: on one
+    # core, and on every core (row slices computed by the single-threaded
+    # oracle in parallel threads)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, n, el = oracle_rate(p, 10.0)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        ncpu, model = cpu_info()
+        gbs1, n1, el1 = oracle_rate(p, 8.0)
+        gbs, n, el = oracle_rate(p, 8.0, threads=ncpu)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": ncpu, "kind": "oracle",
                "sample": f"{n} full {args.config} oracle calls at batch {args.batch} "
-                         f"({el:.1f} s, single thread)"}
+                         f"({el:.1f} s) on {ncpu} row slices in parallel threads",
+               "nproc": ncpu, "cpu_model": model,
+               "single_core": {"value": gbs1, "unit": "GB/s", "cores": 1,
+                               "sample": f"{n1} full calls ({el1:.1f} s, one thread)",
+                               "us_per_call": el1 / n1 * 1e6},
+               "us_per_call": el / n * 1e6}
 
     n_graphs = len(graphs)
     del graphs
@@ -392,17 +469,27 @@ def run_dsq(args):
             "us_per_call": us_call, "frac_of_hbm": achieved / peak,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f16 in / f32 accumulate / f16 out", "data": "synthetic",
-            "config": {"workload": f"{args.config}: {synth.describe(args.config)}",
-                       "batch": args.batch, "rows": p.rows, "cols": p.cols,
-                       "bits": p.bits, "mode": p.mode, "nnz": p.nnz,
-                       "canonical_bytes_per_call": canon,
+            "config": {**gpu_config(args, p, canon),
                        "device_bytes_per_call": per_call,
                        "l2": f"rotating {copies} packed copies "
                              f"({copies * per_call / 1e6:.0f} MB > 2x L2 {l2 / 1e6:.0f} MB)",
                        "timing": f"CUDA events around {n_graphs} CUDA graph replay(s) "
                                  f"of {K} calls"},
+            "us_per_call_dist": {"median": float(np.median(per_replay)),
+                                 "p10": float(np.percentile(per_replay, 10)),
+                                 "p90": float(np.percentile(per_replay, 90)),
+                                 "samples": len(per_replay),
+                                 "what": f"per-call time of each graph replay ({G} calls back to back)"},
+            "isolated_us_per_call": {"median": float(np.median(iso)),
+                                     "p10": float(np.percentile(iso, 10)),
+                                     "p90": float(np.percentile(iso, 90)),
+                                     "samples": len(iso),
+                                     "what": "CUDA events around one call after a device-side "
+                                             "sleep and nothing after it (no overlap with "
+                                             "neighbouring calls, no host launch gap)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
+                         "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_src == "measured" else "fallback 6650 GB/s",
                          "achieved_on_device_bytes": per_call / (us_call * 1e-6) / 1e9,

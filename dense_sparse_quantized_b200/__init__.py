@@ -33,7 +33,7 @@ MODE_AFFINE_G16 = 1
 
 EXPORTS = ("dsq_pack", "dsq_blob_desc", "dsq_create", "dsq_gemv", "dsq_gemv_launches", "dsq_decode",
            "dsq_handle_desc", "dsq_device_bytes", "dsq_check", "dsq_destroy", "dsq_status_string",
-           "dsq_gemv_noalloc")
+           "dsq_gemv_noalloc", "dsq_selftest_wait_timeout")
 
 
 class DSQError(RuntimeError):
@@ -71,6 +71,7 @@ def library() -> ctypes.CDLL:
         lib.dsq_check.argtypes = [P]
         lib.dsq_destroy.argtypes = [P]
         lib.dsq_gemv_noalloc.argtypes = [ctypes.POINTER(Desc), P, SZ, P, P, I, P]
+        lib.dsq_selftest_wait_timeout.argtypes = [P, P]
         lib.dsq_status_string.argtypes = [I]
         lib.dsq_status_string.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -217,6 +218,12 @@ class Handle:
         """Synchronise the device; raise if a kernel of this handle gave up a
         bounded wait since the last check."""
         _check(library().dsq_check(self._h), "dsq_check")
+
+    def selftest_wait_timeout(self, stream=None):
+        """Test hook: launch a kernel whose bounded wait runs out (about 2 s);
+        the next check() raises DSQ_ERR_DEVICE."""
+        _check(library().dsq_selftest_wait_timeout(self._h, _stream_ptr(stream)),
+               "dsq_selftest_wait_timeout")
 
     def close(self):
         if self._h is not None:

@@ -151,6 +151,13 @@ extern "C" int dsq_decode(dsq_handle_t h, void *w_dense_out, void *stream) {
     return launch_decode(h, (__half *)w_dense_out, (cudaStream_t)stream);
 }
 
+extern "C" int dsq_selftest_wait_timeout(dsq_handle_t h, void *stream) {
+    if (!h) return DSQ_ERR_INVALID_ARG;
+    DeviceGuard guard(h->device);
+    if (!guard.ok) return DSQ_ERR_CUDA;
+    return launch_wait_timeout(h, (cudaStream_t)stream);
+}
+
 extern "C" int dsq_handle_desc(dsq_handle_t h, dsq_desc *out) {
     if (!h || !out) return DSQ_ERR_INVALID_ARG;
     out->rows = h->header.rows;

@@ -4,6 +4,7 @@
 // Serves every shape, mode and batch; the tuned kernels replace it on the
 // shapes they cover.  Also dsq_decode's kernel.
 #include "internal.h"
+#include "ptx.h"
 
 namespace dsq {
 
@@ -154,6 +155,24 @@ int launch_decode(const dsq_handle_s *h, __half *w, cudaStream_t st) {
     else if (m.bits == 4 && m.mode == 0) decode_kernel<4, 0><<<grid, threads, 0, st>>>(m, w);
     else if (m.bits == 3) decode_kernel<3, 1><<<grid, threads, 0, st>>>(m, w);
     else decode_kernel<4, 1><<<grid, threads, 0, st>>>(m, w);
+    return cudaGetLastError() == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+}
+
+// One CTA waits on an mbarrier that nothing ever arrives on, through the same
+// bounded wait every pipeline uses; when the wait gives up it records the
+// timeout in the status word and returns.
+__global__ void wait_timeout_kernel(int *status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (!mbar_wait_warp(&bar, 0) && threadIdx.x == 0) report(status, kStatusTimeout);
+}
+
+int launch_wait_timeout(const dsq_handle_s *h, cudaStream_t st) {
+    wait_timeout_kernel<<<1, 32, 0, st>>>(h->d_status);
     return cudaGetLastError() == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
 }
 

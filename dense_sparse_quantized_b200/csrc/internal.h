@@ -83,6 +83,7 @@ int launch_gemv_generic(const dsq_handle_s *h, const __half *x, __half *y, int b
 int launch_decode(const dsq_handle_s *h, __half *w, cudaStream_t stream);
 int gemv_launch_count(const dsq_handle_s *h, int batch);
 int launch_zero(__half *y, int64_t n, cudaStream_t stream);
+int launch_wait_timeout(const dsq_handle_s *h, cudaStream_t stream);
 
 // Tuned batch-1 path (fused_b1.cu).  launch_gemv_fused returns
 // DSQ_ERR_UNSUPPORTED, launching nothing, for shapes it does not cover.

@@ -188,6 +188,18 @@ DSQ_API size_t dsq_device_bytes(dsq_handle_t h);
  */
 DSQ_API int dsq_check(dsq_handle_t h);
 
+/*
+ * dsq_selftest_wait_timeout -- test hook for the failure path of the bounded
+ * waits: launches on `stream` one small kernel that waits on a barrier
+ * nothing ever arrives on, through the same bounded wait (about 2 s) the
+ * product kernels use; the wait gives up, sets the handle's status word and
+ * the kernel returns, leaving the context usable.  A following dsq_check
+ * then returns DSQ_ERR_DEVICE (and clears the word).  No product call makes
+ * such a launch.  Returns DSQ_OK (launched), DSQ_ERR_INVALID_ARG or
+ * DSQ_ERR_CUDA.
+ */
+DSQ_API int dsq_selftest_wait_timeout(dsq_handle_t h, void *stream);
+
 /* dsq_destroy -- free the handle's device memory; NULL is a no-op.  The
  * caller must make sure no work using the handle is still in flight. */
 DSQ_API int dsq_destroy(dsq_handle_t h);

@@ -49,6 +49,7 @@ def test_null_handle_calls_are_rejected_on_the_host():
     assert lib.dsq_destroy(None) == dsq.DSQ_OK
     assert lib.dsq_device_bytes(None) == 0
     assert lib.dsq_create(None, 0, 0, None) == dsq.DSQ_ERR_INVALID_ARG
+    assert lib.dsq_selftest_wait_timeout(None, None) == dsq.DSQ_ERR_INVALID_ARG
 
 
 # --------------------------------------------------------------- validation

@@ -4,6 +4,8 @@ import json
 import os
 import sys
 
+import numpy as np
+
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -60,8 +62,13 @@ def _check_reference_line(line):
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["higher_is_better"] is True and line["dtype"] == "f64"
     assert line["config"]["workload"].startswith("c2:")
+    # the same workload keys as the GPU arm's line
+    for key in ("batch", "rows", "cols", "bits", "mode", "nnz", "canonical_bytes_per_call"):
+        assert key in line["config"], key
+    assert (line["config"]["rows"], line["config"]["cols"], line["config"]["bits"]) == (11008, 4096, 3)
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
+    assert cb["nproc"] >= cb["cores"] and cb["cpu_model"]
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
 
@@ -91,3 +98,24 @@ def test_reference_arm_under_two_ranks_prints_once():
     lines = _json_lines(r.stdout)
     assert len(lines) == 1
     _check_reference_line(lines[0])
+
+
+def test_oracle_rate_threads_cover_every_row_once(monkeypatch):
+    """The all-core CPU baseline runs the unmodified oracle on row slices in
+    threads: together the slices compute exactly the full product."""
+    import oracle
+    import synth
+    p = synth.make_problem(97, 256, 3, "affine", 0.01, "uniform", 3, 1)
+    orc = oracle.load()
+    seen = []
+    real = orc.gemv
+
+    def spy(q, x=None, rows=None):
+        seen.append(np.asarray(rows).copy())
+        return real(q, x=x, rows=rows)
+
+    monkeypatch.setattr(orc, "gemv", spy)
+    gbs, n, el = bench.oracle_rate(p, 0.0, threads=4)
+    assert n == 1 and gbs > 0
+    assert len(seen) == 4
+    assert np.array_equal(np.sort(np.concatenate(seen)), np.arange(p.rows))

@@ -7,6 +7,8 @@ tolerance covers the fp16 rounding of y (<= 2^-11 |y|), the use of exact
 rather than fp16-rounded affine weights inside the group sums (<= 2^-11 per
 weight, i.e. <= 4.9e-4 * bound) and fp32 accumulation.
 """
+import os
+
 import numpy as np
 import pytest
 
@@ -97,14 +99,23 @@ def test_gemv_full_oracle(orc, name, batch):
     check_y(y, y_ref, bound, f"{name} B={batch}")
 
 
+def oracle_all_rows(orc, p, x):
+    """The oracle over every row, computed on row slices in parallel threads
+    (its C entry point releases the GIL); same values as one call."""
+    from concurrent.futures import ThreadPoolExecutor
+    slices = np.array_split(np.arange(p.rows, dtype=np.int32), max(1, min(16, os.cpu_count() or 1)))
+    with ThreadPoolExecutor(max_workers=len(slices)) as pool:
+        parts = list(pool.map(lambda r: orc.gemv(p, x=x, rows=r), slices))
+    return np.concatenate([a for a, _ in parts], axis=1), np.concatenate([b for _, b in parts], axis=1)
+
+
 @pytest.mark.parametrize("name", C4)
 @pytest.mark.parametrize("batch", [1, 16])
-def test_gemv_c4_sampled(orc, name, batch):
+def test_gemv_c4_every_row(orc, name, batch):
     p, h = config(name)
     y = gemv(h, p.x, batch)
-    rows = sample_rows(p, 512)
-    y_ref, bound = orc.gemv(p, x=p.x[:batch], rows=rows)
-    check_y(y[:, rows], y_ref, bound, f"{name} B={batch}")
+    y_ref, bound = oracle_all_rows(orc, p, p.x[:batch])
+    check_y(y, y_ref, bound, f"{name} B={batch}")
 
 
 # ------------------------------------------------------------- small shapes
@@ -361,3 +372,25 @@ def test_wide_range_x_small_affine(orc, rows, cols, per_group, batch):
         y = gemv(h, xb, batch)
     y_ref, bound = orc.gemv(q, x=xb)
     check_y(y, y_ref, bound, f"{rows}x{cols} wide-range per_group={per_group} B={batch}")
+
+
+# ------------------------------------------------------------- bounded waits
+
+def test_bounded_wait_gives_up_reports_and_leaves_the_context_usable(orc):
+    """A kernel waits on a barrier nothing arrives on, through the bounded wait
+    every pipeline uses: after about 2 s it gives up and sets the status word;
+    dsq_check reports DSQ_ERR_DEVICE once and clears it; the next product on
+    the same handle is correct and checks clean."""
+    import time
+    p = synth.make_problem(64, 512, 3, "affine", 0.01, "uniform", 11, 1)
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        t0 = time.perf_counter()
+        h.selftest_wait_timeout()
+        with pytest.raises(dsq.DSQError) as e:
+            h.check()
+        assert e.value.status == dsq.DSQ_ERR_DEVICE
+        assert time.perf_counter() - t0 >= 1.0   # the wait ran to its limit
+        h.check()                                 # the word was cleared
+        y = gemv(h, p.x, 1)
+        y_ref, bound = orc.gemv(p)
+        check_y(y, y_ref, bound, "after a timed-out wait")

@@ -56,10 +56,12 @@ def random_x(seed, batch, cols):
     return synth.f16_bits(rng.standard_normal((batch, cols)))
 
 
-# Two affine 3-bit matrices whose K splits differ (2000 rows: 16 tiles, a
-# 4-way split; 6000 rows: 47 tiles, a 3-way split), so the second call must
-# not reuse the first one's split starts.
-CASES = [(2000, 4096, 0.01, "topk", 24), (6000, 2048, 0.005, "zipf", 80)]
+# Affine 3-bit matrices with different row counts, so consecutive calls leave
+# different contents in the shared scratch: 2000 rows (16 tiles of 128 rows)
+# and 6000 rows (47 tiles) both get a 2-way K split (two CTAs per tile fit the
+# 148 SMs) with different split starts; 10000 rows (79 tiles) get none, the
+# path that only clears the status word.
+CASES = [(2000, 4096, 0.01, "topk", 24), (6000, 2048, 0.005, "zipf", 80), (10000, 1024, 0.01, "uniform", 16)]
 
 
 def test_two_calls_in_a_row_match_dsq_gemv(orc):
@@ -68,7 +70,7 @@ def test_two_calls_in_a_row_match_dsq_gemv(orc):
         p = synth.make_problem(rows, cols, 3, "affine", dens, kind, 900 + i, 1)
         blob = dsq.pack_problem(p)
         mats.append((p, blob, dsq.blob_desc(blob), upload(blob), dsq.Handle(blob), batch))
-    calls = [(0, 11), (1, 12), (1, 13), (0, 14)]
+    calls = [(0, 11), (1, 12), (1, 13), (2, 15), (0, 14), (2, 16)]
     for m, seed in calls:
         p, blob, desc, dev_blob, h, batch = mats[m]
         xb = random_x(seed, batch, p.cols)
