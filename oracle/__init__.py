@@ -7,7 +7,8 @@ older than the source, or takes another source file (tests compile planted
 mistakes that way, into a temporary directory).
 
 Each function takes a problem object with the attributes ``rows, cols, bits,
-mode ('lut' | 'affine'), codes, table, zeros, row_ptr, col_idx, values`` as
+mode ('lut' | 'affine' | 'bitplane'), codes, table, zeros, row_ptr, col_idx,
+values`` as
 numpy arrays of the dtypes the synthetic generator produces.
 """
 from __future__ import annotations
@@ -72,7 +73,7 @@ class Oracle:
     # -- the method ----------------------------------------------------
     @staticmethod
     def _args(p):
-        mode = 0 if p.mode == "lut" else 1
+        mode = {"lut": 0, "affine": 1, "bitplane": 2}[p.mode]
         codes = np.ascontiguousarray(p.codes, dtype=np.uint8)
         table = np.ascontiguousarray(p.table, dtype=np.uint16)
         zeros = (np.ascontiguousarray(p.zeros, dtype=np.uint16)

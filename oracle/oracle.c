@@ -23,6 +23,12 @@
  *  - SqueezeLLM page, "Sensitivity-based non-uniform quantization": the dense
  *    part is codes into a non-uniform table of bins; read as one fp16 table
  *    of 2^bits centroids per output row, w = table[row][q].
+ *  - BPDQ page, "1. Formulation de la Grille Variable": the dense part is
+ *    What = REP(C_0) + sum_{i=1..k} REP(C_i) (.) B_i, with k bit planes
+ *    B_i in {0,1} and scalar coefficients C_0..C_k per group along the input
+ *    dimension.  Read as: groups of 32 * 2^k inputs, fp16 coefficients, a
+ *    weight's k plane bits held in one code q with b_i = bit (i-1) of q, and
+ *    the sum C_0 + sum_i C_i b_i evaluated exactly and rounded once to fp16.
  *
  * Precision.  A decoded dense weight is an fp16 value: a table entry is
  * copied bit for bit; an affine weight is scale*(q-zero) evaluated exactly in
@@ -43,6 +49,7 @@
 
 #define ORACLE_LUT 0
 #define ORACLE_AFFINE 1
+#define ORACLE_BITPLANE 2
 #define ORACLE_GROUP 16
 
 /* IEEE 754 binary16 -> real value: sign, 5-bit biased exponent (bias 15),
@@ -111,8 +118,9 @@ void oracle_double_to_half_n(const double *v, uint16_t *out, int64_t n)
 }
 
 /* Decoded dense weight of row i, column j, as an fp16 bit pattern.
- * table: LUT mode rows x 2^bits centroids; AFFINE mode rows x cols/16 scales.
- * zeros: AFFINE mode rows x cols/16 integral zeros (unused in LUT mode). */
+ * table: LUT mode rows x 2^bits centroids; AFFINE mode rows x cols/16 scales;
+ * BITPLANE mode rows x cols/(32*2^bits) x (bits+1) coefficients C_0..C_k.
+ * zeros: AFFINE mode rows x cols/16 integral zeros (unused otherwise). */
 uint16_t oracle_decode_one(int64_t i, int64_t j, int cols, int bits, int mode,
                            const uint8_t *codes, const uint16_t *table,
                            const uint16_t *zeros)
@@ -120,6 +128,17 @@ uint16_t oracle_decode_one(int64_t i, int64_t j, int cols, int bits, int mode,
     int q = codes[i * (int64_t)cols + j];
     if (mode == ORACLE_LUT)
         return table[i * ((int64_t)1 << bits) + q];
+    if (mode == ORACLE_BITPLANE) {
+        /* C_0 + sum over the planes whose bit is set; fp16 terms of at most
+         * 11 significant bits between 2^-24 and 2^16 sum exactly in fp64 */
+        int64_t gsize = (int64_t)32 << bits;
+        const uint16_t *c = table + (i * (cols / gsize) + j / gsize) * (bits + 1);
+        double w = oracle_half_to_double(c[0]);
+        for (int p = 1; p <= bits; p++)
+            if ((q >> (p - 1)) & 1)
+                w += oracle_half_to_double(c[p]);
+        return oracle_double_to_half(w);
+    }
     {
         int64_t g = i * (int64_t)(cols / ORACLE_GROUP) + j / ORACLE_GROUP;
         double scale = oracle_half_to_double(table[g]);

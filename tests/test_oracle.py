@@ -58,6 +58,9 @@ def random_problem(rng, rows, cols, bits, mode, batch, nnz_per_row_max=4,
     if mode == "lut":
         table = random_finite_f16(rng, (rows, K), -20, 4)
         zeros = None
+    elif mode == "bitplane":
+        table = random_finite_f16(rng, (rows, cols // (32 << bits), bits + 1), -12, 2)
+        zeros = None
     else:
         table = random_finite_f16(rng, (rows, cols // 16), *scale_exp)
         zeros = np_d2h(rng.integers(0, K, size=(rows, cols // 16)))
@@ -169,6 +172,65 @@ def pin_affine_group_layout(orc):
     assert np.array_equal(np_h2d(orc.decode(p)), want)
 
 
+def bp_group(k):
+    """Inputs per coefficient group of a bit-plane matrix with k planes."""
+    return 32 << k
+
+
+def pin_bitplane_decode_golden(orc):
+    """Hand-worked C0 + sum_i C_i b_i values (BPDQ page, "Formulation de la
+    Grille Variable"): plane order, ties, subnormals, overflow, and one
+    rounding of the exact sum rather than one per addition."""
+    g = json.load(open(os.path.join(GOLDEN, "bitplane_decode.json")))
+    for c in g["cases"]:
+        k = c["k"]
+        K, G = 1 << k, bp_group(k)
+        codes = np.tile(np.arange(K), G // K)
+        coef = [[[int(v, 16) for v in c["coef"]]]]
+        p = problem(1, G, k, "bitplane", codes, coef, None, [0, 0], [], [], np.zeros(G))
+        got = orc.decode(p)[0]
+        want = np.array([int(v, 16) for v in c["expect"]], np.uint16)
+        assert np.array_equal(got, np.tile(want, G // K)), (c["why"], [hex(int(v)) for v in got[:K]])
+
+
+def pin_bitplane_group_layout(orc):
+    """Group g of row r covers columns g*32*2^k .. (g+1)*32*2^k - 1 and has
+    its own coefficients; with C0 = 10 r + g, C1 = 1, C2 = 2 (, C3 = 4) the
+    weight is the integer C0 + q."""
+    for k in (2, 3):
+        G, K = bp_group(k), 1 << k
+        cols = 2 * G
+        codes = np.tile(np.arange(cols) % K, (2, 1))
+        coef = np.zeros((2, 2, k + 1))
+        for r in range(2):
+            for g in range(2):
+                coef[r, g] = [10 * r + g] + [2.0 ** i for i in range(k)]
+        p = problem(2, cols, k, "bitplane", codes, np_d2h(coef), None, [0, 0, 0], [], [], np.zeros(cols))
+        grp = np.arange(cols) // G
+        want = np.stack([10 * r + grp + np.arange(cols) % K for r in range(2)]).astype(np.float64)
+        assert np.array_equal(np_h2d(orc.decode(p)), want)
+
+
+def pin_bitplane_uniform_grid_is_affine(orc):
+    """A bit-plane group with C_i = s * 2^(i-1) and C0 = -s * z is the
+    uniform grid s * (q - z): it decodes exactly as the (separately pinned)
+    affine decode with scale s and zero z, for every code."""
+    rng = np.random.default_rng(21)
+    for k in (2, 3):
+        G, K = bp_group(k), 1 << k
+        for _ in range(20):
+            m = int(rng.integers(1, 128))              # <= 7 significant bits: s * z stays exact
+            e = int(rng.integers(-20, 4))
+            s = m * 2.0 ** e
+            z = int(rng.integers(0, K))
+            coef = [[np_d2h([0.0 - s * z] + [s * 2.0 ** i for i in range(k)])]]   # +0 when z = 0
+            codes = np.tile(np.arange(K), G // K)
+            bp = problem(1, G, k, "bitplane", codes, coef, None, [0, 0], [], [], np.zeros(G))
+            af = problem(1, G, 3, "affine", codes, np.full((1, G // 16), np_d2h(s)),
+                         np.full((1, G // 16), np_d2h(float(z))), [0, 0], [], [], np.zeros(G))
+            assert np.array_equal(orc.decode(bp), orc.decode(af)), (k, s, z)
+
+
 # ------------------------------------------------------------------ product pins
 
 def exact_reference(p):
@@ -181,6 +243,11 @@ def exact_reference(p):
             q = int(p.codes[i, j])
             if p.mode == "lut":
                 W[i][j] = Fraction(float(np_h2d(p.table[i, q])))
+            elif p.mode == "bitplane":
+                G = 32 << p.bits
+                c = [Fraction(float(v)) for v in np_h2d(p.table[i, j // G])]
+                exact = c[0] + sum(c[t] for t in range(1, p.bits + 1) if (q >> (t - 1)) & 1)
+                W[i][j] = Fraction(float(np_h2d(np_d2h(float(exact)))))
             else:
                 s = Fraction(float(np_h2d(p.table[i, j // 16])))
                 z = Fraction(float(np_h2d(p.zeros[i, j // 16])))
@@ -200,8 +267,9 @@ def pin_gemv_exact(orc):
     summation bound (n+2) * 2^-52 * bound, on small random problems of both
     modes and code widths, several rows, a batch of 3 and scattered outliers."""
     rng = np.random.default_rng(5)
-    for bits, mode in ((3, "lut"), (4, "lut"), (3, "affine"), (4, "affine")):
-        p = random_problem(rng, 5, 32, bits, mode, 3)
+    for bits, mode, cols in ((3, "lut", 32), (4, "lut", 32), (3, "affine", 32), (4, "affine", 32),
+                             (2, "bitplane", 256), (3, "bitplane", 256)):
+        p = random_problem(rng, 5, cols, bits, mode, 3)
         y, bd = orc.gemv(p)
         ye, be = exact_reference(p)
         tol = (p.cols + 2) * 2.0 ** -52
@@ -269,6 +337,7 @@ def pin_rows_subset(orc):
 
 PINS = [pin_half_to_double_exhaustive, pin_double_to_half, pin_csr_example,
         pin_lut_decode_identity, pin_affine_decode_golden, pin_affine_group_layout,
+        pin_bitplane_decode_golden, pin_bitplane_group_layout, pin_bitplane_uniform_grid_is_affine,
         pin_gemv_exact, pin_special_cases, pin_decomposition, pin_rows_subset]
 
 
@@ -302,6 +371,13 @@ MUTANTS = {
     "x_transposed": ("acc += wrow[j] * xd[(int64_t)b * cols + j];",
                      "acc += wrow[j] * xd[(int64_t)j * batch + b];"),
     "dropped_x": ("acc += wrow[j] * xd[(int64_t)b * cols + j];", "acc += wrow[j];"),
+    "bitplane_bit_order": ("if ((q >> (p - 1)) & 1)", "if ((q >> p) & 1)"),
+    "bitplane_drop_bias": ("double w = oracle_half_to_double(c[0]);", "double w = 0.0;"),
+    "bitplane_group_size": ("int64_t gsize = (int64_t)32 << bits;", "int64_t gsize = (int64_t)16 << bits;"),
+    "bitplane_round_each_step": ("                w += oracle_half_to_double(c[p]);",
+                                 "                w = oracle_half_to_double(oracle_double_to_half(w + oracle_half_to_double(c[p])));"),
+    "bitplane_coef_row_stride": ("table + (i * (cols / gsize) + j / gsize) * (bits + 1)",
+                                 "table + (j / gsize) * (bits + 1)"),
     "first_column_skipped": ("for (int64_t j = 0; j < cols; j++) {\n                acc",
                              "for (int64_t j = 1; j < cols; j++) {\n                acc"),
 }
