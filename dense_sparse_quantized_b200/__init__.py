@@ -30,6 +30,7 @@ DSQ_ERR_DEVICE = -6
 DSQ_ERR_SCRATCH_LIMIT = -7
 MODE_LUT_ROW = 0
 MODE_AFFINE_G16 = 1
+MODE_BITPLANE = 2
 
 EXPORTS = ("dsq_pack", "dsq_blob_desc", "dsq_create", "dsq_gemv", "dsq_gemv_launches", "dsq_decode",
            "dsq_handle_desc", "dsq_device_bytes", "dsq_check", "dsq_destroy", "dsq_status_string",
@@ -101,12 +102,13 @@ def pack(rows: int, cols: int, bits: int, mode, codes, table, zeros, row_ptr, co
          values) -> bytes:
     """Validate logical weights and return the packed blob (host bytes).
 
-    mode: 'lut' / 'affine' or MODE_LUT_ROW / MODE_AFFINE_G16.  Arrays: codes
-    uint8 [rows, cols]; table fp16 bits (uint16) [rows, 2^bits] or
-    [rows, cols/16]; zeros uint16 [rows, cols/16] or None; row_ptr int32;
-    col_idx int32; values uint16 fp16 bits."""
+    mode: 'lut' / 'affine' / 'bitplane' or MODE_*.  Arrays: codes uint8
+    [rows, cols]; table fp16 bits (uint16) [rows, 2^bits] (lut),
+    [rows, cols/16] (affine scales) or [rows, cols/(32*2^bits), bits+1]
+    (bit-plane coefficients C0..Ck); zeros uint16 [rows, cols/16] or None;
+    row_ptr int32; col_idx int32; values uint16 fp16 bits."""
     lib = library()
-    m = {"lut": MODE_LUT_ROW, "affine": MODE_AFFINE_G16}.get(mode, mode)
+    m = {"lut": MODE_LUT_ROW, "affine": MODE_AFFINE_G16, "bitplane": MODE_BITPLANE}.get(mode, mode)
     nnz = int(np.asarray(row_ptr)[-1]) if row_ptr is not None and len(row_ptr) else 0
     d = Desc(int(rows), int(cols), int(bits), int(m), nnz)
     keep = [_arr(codes, np.uint8), _arr(table, np.uint16), _arr(zeros, np.uint16),

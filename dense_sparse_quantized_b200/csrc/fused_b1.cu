@@ -1,5 +1,6 @@
-// fused_b1.cu -- batch-1 dense+sparse GEMV: 3-bit affine group-16 rows and
-// 3/4-bit row-LUT rows, one pass, y written once.
+// fused_b1.cu -- batch-1 dense+sparse GEMV: 3-bit affine group-16 rows,
+// 3/4-bit row-LUT rows and 2/3-bit-plane rows (per-group level tables), one
+// pass, y written once; and the table kernel for 2-4 activation rows.
 //
 // One CTA per row tile (contiguous rows of about equal cost, one tile per
 // SM, from a host schedule built at create).  Warp (rg, cw) owns slot
@@ -270,11 +271,19 @@ __device__ __forceinline__ float decode_aff3(const uint4 v, uint32_t zb, const u
     return fmaf(sB, acc[1][0] + acc[1][1], sA * (acc[0][0] + acc[0][1]));
 }
 
-// Table slot: code words w[0..BITS-1], this row's centroid held by the lane.
+// Table slot: code words w[0..BITS-1], the table entry held by the lane (a
+// centroid of the row, or a level of the lane's bit-plane group).
 template <int BITS>
 __device__ __forceinline__ float decode_lut(const uint32_t (&w)[4], float tv, const float (&xr)[32]) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (BITS == 4) {
+    if (BITS == 2) {
+#pragma unroll
+        for (int c = 0; c < 32; c++) {
+            const uint32_t wd = w[c >> 4];
+            const int sh = 2 * (c & 15);
+            acc[c & 3] = fmaf(__shfl_sync(kFull, tv, sh ? (int)(wd >> sh) : (int)wd, 4), xr[c], acc[c & 3]);
+        }
+    } else if (BITS == 4) {
 #pragma unroll
         for (int c = 0; c < 32; c++) {
             const uint32_t wd = w[c >> 3];
@@ -494,10 +503,14 @@ b1_aff3_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y)
     finalize(td, smem, p, 1.0f, y);
 }
 
-template <int KIND>  // 3: LUT 3-bit, 4: LUT 4-bit
+// Table lookup by shfl.idx over 2^BITS-lane segments.  Row tables (GT
+// false): every segment holds the row's 2^BITS centroids.  Bit-plane groups
+// (GT true): a group spans 2^BITS slots, i.e. exactly one segment, whose lanes
+// hold that group's 2^BITS levels -- the lane of slot s holds level s % 2^BITS
+// of group s / 2^BITS -- so the same lookup reads the lane's own group.
+template <int BITS, bool GT>
 __global__ void __launch_bounds__(kThreads, 1)
 b1_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) {
-    constexpr int BITS = KIND == 4 ? 4 : 3;
     constexpr int K = 1 << BITS;
     constexpr int NW = BITS;  // 32-bit code words per slot and row
     extern __shared__ __align__(128) unsigned char smem[];
@@ -519,8 +532,10 @@ b1_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) 
     const size_t row_step = (size_t)R * m.row_words * 4;
     const unsigned char *rec = reinterpret_cast<const unsigned char *>(m.dense) +
                                ((size_t)td.r0 + rg) * m.row_words * 4;
+    const int te = GT ? min(s, S - 1) : (lane & (K - 1));  // this lane's entry of the row's table
     const unsigned char *tabp = reinterpret_cast<const unsigned char *>(m.table) +
-                                ((size_t)(td.r0 + rg) * K + (lane & (K - 1))) * 2 - 2 * (lane & 1);
+                                ((size_t)(td.r0 + rg) * (GT ? S : K) + te) * 2 - 2 * (te & 1);
+    const size_t tab_step = (size_t)R * (GT ? S : K) * 2;
     const int nj = rg < nrows ? (nrows - rg + R - 1) / R : 0;
     int issued = 0;
     auto issue = [&](int d) {
@@ -534,10 +549,10 @@ b1_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) 
                     for (int k = 0; k < NW; k++) cp_async4(st + 4 * k, rec + 4 * ((size_t)k * S + s));
                 }
             }
-            // the 4-byte word holding this lane's centroid (table rows are 16/32-byte aligned)
+            // the 4-byte word holding this lane's entry (table rows are 4-byte aligned)
             cp_async4(sa, tabp);
             rec += row_step;
-            tabp += (size_t)R * K * 2;
+            tabp += tab_step;
         }
         issued++;
         cp_async_commit();
@@ -578,7 +593,7 @@ b1_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) 
                     for (int k = 0; k < NW; k++) w4[k] = lds32(st + 4 * k);
                 }
             }
-            const float tv = __half2float(__ushort_as_half((unsigned short)(lds32(sa) >> (16 * (lane & 1)))));
+            const float tv = __half2float(__ushort_as_half((unsigned short)(lds32(sa) >> (16 * (te & 1)))));
             float r = decode_lut<BITS>(w4, tv, xr);
             r = warp_sum(r);
             if (lane == 0) part[(size_t)i * C + cw] = r;
@@ -601,7 +616,7 @@ constexpr int kThreadsN = kMaxWarpsN * 32;
 // every activation row as fp16 pairs, looks each weight up once (shfl.idx,
 // fp16 centroid) and adds weight * x for every row with mixed-precision
 // FMAs.  Outliers: one lane per piece after the dense loop, x read from L2.
-template <int BITS, int NB>
+template <int BITS, bool GT, int NB>
 __global__ void __launch_bounds__(kThreadsN, 1)
 bn_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y, int nb) {
     constexpr int K = 1 << BITS;
@@ -621,8 +636,10 @@ bn_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y, 
     const size_t row_step = (size_t)R * m.row_words * 4;
     const unsigned char *rec = reinterpret_cast<const unsigned char *>(m.dense) +
                                ((size_t)td.r0 + rg) * m.row_words * 4;
+    const int te = GT ? min(s, S - 1) : (lane & (K - 1));  // as in b1_lut_kernel
     const unsigned char *tabp = reinterpret_cast<const unsigned char *>(m.table) +
-                                ((size_t)(td.r0 + rg) * K + (lane & (K - 1))) * 2 - 2 * (lane & 1);
+                                ((size_t)(td.r0 + rg) * (GT ? S : K) + te) * 2 - 2 * (te & 1);
+    const size_t tab_step = (size_t)R * (GT ? S : K) * 2;
     const int nj = rg < nrows ? (nrows - rg + R - 1) / R : 0;
     int issued = 0;
     auto issue = [&](int d) {
@@ -638,7 +655,7 @@ bn_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y, 
             }
             cp_async4(sa, tabp);
             rec += row_step;
-            tabp += (size_t)R * K * 2;
+            tabp += tab_step;
         }
         issued++;
         cp_async_commit();
@@ -682,15 +699,18 @@ bn_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y, 
                 for (int k = 0; k < NW; k++) w4[k] = lds32(st + 4 * k);
             }
         }
-        // this lane's centroid as fp16 bits (the word holds two entries)
-        const uint32_t tv = (lds32(sa) >> (16 * (lane & 1))) & 0xffffu;
+        // this lane's table entry as fp16 bits (the word holds two entries)
+        const uint32_t tv = (lds32(sa) >> (16 * (te & 1))) & 0xffffu;
         float lo[NB], hi[NB];
 #pragma unroll
         for (int b = 0; b < NB; b++) lo[b] = hi[b] = 0.f;
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
             int q0, q1;
-            if (BITS == 4) {
+            if (BITS == 2) {
+                q0 = (int)(w4[c >> 4] >> (2 * (c & 15)));
+                q1 = (int)(w4[c >> 4] >> (2 * ((c + 1) & 15)));
+            } else if (BITS == 4) {
                 q0 = (int)(w4[c >> 3] >> (4 * (c & 7)));
                 q1 = (int)(w4[c >> 3] >> (4 * ((c + 1) & 7)));
             } else if (c < 30) {
@@ -785,12 +805,13 @@ bn_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y, 
     }
 }
 
-enum Kind { kNone = -1, kAff3 = 0, kLut3 = 3, kLut4 = 4 };
+enum Kind { kNone = -1, kAff3 = 0, kLut3 = 3, kLut4 = 4, kBp2 = 12, kBp3 = 13 };
 
 Kind b1_kind(const MatrixView &m, int batch) {
     if (batch != 1 || m.rows <= 0 || m.cols <= 0) return kNone;
     if ((m.slots + 31) / 32 > kMaxWarps) return kNone;
     if (m.mode == DSQ_MODE_AFFINE_G16) return m.bits == 3 ? kAff3 : kNone;
+    if (m.mode == DSQ_MODE_BITPLANE) return m.bits == 2 ? kBp2 : kBp3;
     return m.bits == 3 ? kLut3 : kLut4;
 }
 
@@ -975,12 +996,18 @@ void free_schedule(dsq_handle_s *h) {
 int fused_prepare(dsq_handle_s *) {
     int rc = set_smem_attr(b1_aff3_kernel<kThreads, 1>);
     if (rc == DSQ_OK) rc = set_smem_attr(b1_aff3_kernel<kWarps2 * 32, 2>);
-    if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<kLut3>);
-    if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<kLut4>);
-    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<3, 2>);
-    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<3, 4>);
-    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<4, 2>);
-    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<4, 4>);
+    if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<3, false>);
+    if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<4, false>);
+    if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<2, true>);
+    if (rc == DSQ_OK) rc = set_smem_attr(b1_lut_kernel<3, true>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<3, false, 2>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<3, false, 4>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<4, false, 2>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<4, false, 4>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<2, true, 2>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<2, true, 4>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<3, true, 2>);
+    if (rc == DSQ_OK) rc = set_smem_attr(bn_lut_kernel<3, true, 4>);
     return rc;
 }
 
@@ -991,7 +1018,7 @@ int batched_launch_count(const dsq_handle_s *h, int batch) {
     B1Params p;
     size_t smem;
     const MatrixView &m = h->view;
-    if (batch < 2 || m.mode != DSQ_MODE_LUT_ROW || m.rows <= 0 || m.cols <= 0 || h->sched.n_tiles == 0 ||
+    if (batch < 2 || m.mode == DSQ_MODE_AFFINE_G16 || m.rows <= 0 || m.cols <= 0 || h->sched.n_tiles == 0 ||
         !plan_bn(h, 4, &p, &smem))
         return -1;
     return (batch + 3) / 4;
@@ -1019,12 +1046,18 @@ int launch_gemv_batched(const dsq_handle_s *h, const __half *x, __half *y, int b
         const __half *xb = x + (size_t)b0 * m.cols;
         __half *yb = y + (size_t)b0 * m.rows;
         cudaError_t e;
-        if (m.bits == 3)
-            e = NB == 2 ? cudaLaunchKernelEx(&cfg, bn_lut_kernel<3, 2>, p, xb, yb, nb)
-                        : cudaLaunchKernelEx(&cfg, bn_lut_kernel<3, 4>, p, xb, yb, nb);
+        if (m.mode == DSQ_MODE_BITPLANE && m.bits == 2)
+            e = NB == 2 ? cudaLaunchKernelEx(&cfg, bn_lut_kernel<2, true, 2>, p, xb, yb, nb)
+                        : cudaLaunchKernelEx(&cfg, bn_lut_kernel<2, true, 4>, p, xb, yb, nb);
+        else if (m.mode == DSQ_MODE_BITPLANE)
+            e = NB == 2 ? cudaLaunchKernelEx(&cfg, bn_lut_kernel<3, true, 2>, p, xb, yb, nb)
+                        : cudaLaunchKernelEx(&cfg, bn_lut_kernel<3, true, 4>, p, xb, yb, nb);
+        else if (m.bits == 3)
+            e = NB == 2 ? cudaLaunchKernelEx(&cfg, bn_lut_kernel<3, false, 2>, p, xb, yb, nb)
+                        : cudaLaunchKernelEx(&cfg, bn_lut_kernel<3, false, 4>, p, xb, yb, nb);
         else
-            e = NB == 2 ? cudaLaunchKernelEx(&cfg, bn_lut_kernel<4, 2>, p, xb, yb, nb)
-                        : cudaLaunchKernelEx(&cfg, bn_lut_kernel<4, 4>, p, xb, yb, nb);
+            e = NB == 2 ? cudaLaunchKernelEx(&cfg, bn_lut_kernel<4, false, 2>, p, xb, yb, nb)
+                        : cudaLaunchKernelEx(&cfg, bn_lut_kernel<4, false, 4>, p, xb, yb, nb);
         if (e != cudaSuccess) return DSQ_ERR_CUDA;
     }
     return DSQ_OK;
@@ -1060,8 +1093,10 @@ int launch_gemv_fused(const dsq_handle_s *h, const __half *x, __half *y, int bat
             e = h->sched.per_sm == 2 ? cudaLaunchKernelEx(&cfg, b1_aff3_kernel<kWarps2 * 32, 2>, p, x, y)
                                      : cudaLaunchKernelEx(&cfg, b1_aff3_kernel<kThreads, 1>, p, x, y);
             break;
-        case kLut3: e = cudaLaunchKernelEx(&cfg, b1_lut_kernel<kLut3>, p, x, y); break;
-        default: e = cudaLaunchKernelEx(&cfg, b1_lut_kernel<kLut4>, p, x, y); break;
+        case kLut3: e = cudaLaunchKernelEx(&cfg, b1_lut_kernel<3, false>, p, x, y); break;
+        case kBp2: e = cudaLaunchKernelEx(&cfg, b1_lut_kernel<2, true>, p, x, y); break;
+        case kBp3: e = cudaLaunchKernelEx(&cfg, b1_lut_kernel<3, true>, p, x, y); break;
+        default: e = cudaLaunchKernelEx(&cfg, b1_lut_kernel<4, false>, p, x, y); break;
     }
     return e == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
 }

@@ -1,5 +1,6 @@
 // generic.cu -- the reference-quality CUDA path: one warp per output row,
-// every weight decoded to its fp16 value exactly as dsq_decode writes it,
+// every weight decoded to its fp16 value exactly as dsq_decode writes it
+// (table entry, fp16(scale * (q - zero)), or the bit-plane group level),
 // fp32 accumulation, CSR outliers added by the same warp, y written once.
 // Serves every shape, mode and batch; the tuned kernels replace it on the
 // shapes they cover.  Also dsq_decode's kernel.
@@ -32,17 +33,27 @@ __device__ __forceinline__ void load_slot(const MatrixView &m, const uint32_t *r
     }
 }
 
-// fp16 value of the decoded dense weight (bits as an unsigned short).
-template <int MODE>
+// fp16 value of the decoded dense weight of column c of slot s.  row_table:
+// the row's centroids (LUT_ROW) or its per-group levels (BITPLANE: the 2^BITS
+// levels of every group of 2^BITS slots, one after the other).
+template <int BITS, int MODE>
 __device__ __forceinline__ __half decode_weight(const __half *row_table, uint32_t q,
-                                                uint32_t scales, uint32_t zb, int c) {
+                                                uint32_t scales, uint32_t zb, int c, int s) {
     if (MODE == DSQ_MODE_LUT_ROW) return row_table[q];
+    if (MODE == DSQ_MODE_BITPLANE) return row_table[((s >> BITS) << BITS) + q];
     int e = c >> 4;  // group inside the slot
-    __half s = __ushort_as_half((unsigned short)(scales >> (16 * e)));
+    __half sc = __ushort_as_half((unsigned short)(scales >> (16 * e)));
     int z = (int)((zb >> (4 * e)) & 15u);
-    // (q - z) is a small integer and s has an 11-bit significand: the fp32
-    // product is exact, so this is the single rounding of s*(q-z) to fp16.
-    return __float2half_rn(__half2float(s) * (float)((int)q - z));
+    // (q - z) is a small integer and sc has an 11-bit significand: the fp32
+    // product is exact, so this is the single rounding of sc*(q-z) to fp16.
+    return __float2half_rn(__half2float(sc) * (float)((int)q - z));
+}
+
+template <int BITS, int MODE>
+__device__ __forceinline__ const __half *row_table_of(const MatrixView &m, int row) {
+    if (MODE == DSQ_MODE_LUT_ROW) return (const __half *)m.table + ((size_t)row << BITS);
+    if (MODE == DSQ_MODE_BITPLANE) return (const __half *)m.table + (size_t)row * m.slots;
+    return nullptr;
 }
 
 template <int BITS, int MODE, int BC>
@@ -54,7 +65,7 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(MatrixView m, const _
     const int nb = min(BC, batch - b0);
     const int N = m.cols;
     const uint32_t *rec = m.dense + (size_t)row * m.row_words;
-    const __half *row_table = MODE == DSQ_MODE_LUT_ROW ? (const __half *)m.table + ((size_t)row << BITS) : nullptr;
+    const __half *row_table = row_table_of<BITS, MODE>(m, row);
     float acc[BC];
 #pragma unroll
     for (int b = 0; b < BC; b++) acc[b] = 0.f;
@@ -66,7 +77,7 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(MatrixView m, const _
         for (int c = 0; c < 32; c++) {
             const int j = s * 32 + c;
             if (j < N) {
-                float wv = __half2float(decode_weight<MODE>(row_table, slot_code<BITS>(w, c), scales, zb, c));
+                float wv = __half2float(decode_weight<BITS, MODE>(row_table, slot_code<BITS>(w, c), scales, zb, c, s));
 #pragma unroll
                 for (int b = 0; b < BC; b++)
                     if (b < nb) acc[b] = fmaf(wv, __half2float(x[(size_t)(b0 + b) * N + j]), acc[b]);
@@ -97,14 +108,14 @@ __global__ void decode_kernel(MatrixView m, __half *__restrict__ w_out) {
     if (t >= (int64_t)m.rows * m.slots) return;
     const int row = (int)(t / m.slots), s = (int)(t % m.slots);
     const uint32_t *rec = m.dense + (size_t)row * m.row_words;
-    const __half *row_table = MODE == DSQ_MODE_LUT_ROW ? (const __half *)m.table + ((size_t)row << BITS) : nullptr;
+    const __half *row_table = row_table_of<BITS, MODE>(m, row);
     uint32_t w[4] = {0, 0, 0, 0}, scales = 0, zb = 0;
     load_slot<BITS, MODE>(m, rec, s, w, scales, zb);
 #pragma unroll
     for (int c = 0; c < 32; c++) {
         const int j = s * 32 + c;
         if (j < m.cols)
-            w_out[(size_t)row * m.cols + j] = decode_weight<MODE>(row_table, slot_code<BITS>(w, c), scales, zb, c);
+            w_out[(size_t)row * m.cols + j] = decode_weight<BITS, MODE>(row_table, slot_code<BITS>(w, c), scales, zb, c, s);
     }
 }
 
@@ -132,7 +143,10 @@ int launch_gemv_generic(const dsq_handle_s *h, const __half *x, __half *y, int b
     const MatrixView &m = h->view;
     if (m.rows == 0) return DSQ_OK;
     if (m.cols == 0) return launch_zero(y, (int64_t)batch * m.rows, st);
-    if (m.bits == 3 && m.mode == 0) launch_generic_t<3, 0>(m, x, y, batch, st);
+    if (m.mode == DSQ_MODE_BITPLANE) {
+        if (m.bits == 2) launch_generic_t<2, 2>(m, x, y, batch, st);
+        else launch_generic_t<3, 2>(m, x, y, batch, st);
+    } else if (m.bits == 3 && m.mode == 0) launch_generic_t<3, 0>(m, x, y, batch, st);
     else if (m.bits == 4 && m.mode == 0) launch_generic_t<4, 0>(m, x, y, batch, st);
     else if (m.bits == 3) launch_generic_t<3, 1>(m, x, y, batch, st);
     else launch_generic_t<4, 1>(m, x, y, batch, st);
@@ -151,7 +165,10 @@ int launch_decode(const dsq_handle_s *h, __half *w, cudaStream_t st) {
     if (n == 0) return DSQ_OK;
     const int threads = 256;
     const unsigned grid = (unsigned)((n + threads - 1) / threads);
-    if (m.bits == 3 && m.mode == 0) decode_kernel<3, 0><<<grid, threads, 0, st>>>(m, w);
+    if (m.mode == DSQ_MODE_BITPLANE) {
+        if (m.bits == 2) decode_kernel<2, 2><<<grid, threads, 0, st>>>(m, w);
+        else decode_kernel<3, 2><<<grid, threads, 0, st>>>(m, w);
+    } else if (m.bits == 3 && m.mode == 0) decode_kernel<3, 0><<<grid, threads, 0, st>>>(m, w);
     else if (m.bits == 4 && m.mode == 0) decode_kernel<4, 0><<<grid, threads, 0, st>>>(m, w);
     else if (m.bits == 3) decode_kernel<3, 1><<<grid, threads, 0, st>>>(m, w);
     else decode_kernel<4, 1><<<grid, threads, 0, st>>>(m, w);

@@ -3,7 +3,10 @@
 // The blob is a 256-byte header followed by 256-byte-aligned sections:
 //
 //   dense    rows x row_words u32: one "row record" per output row
-//   table    LUT_ROW only: rows x 2^bits fp16 centroids, as given
+//   table    LUT_ROW: rows x 2^bits fp16 centroids, as given;
+//            BITPLANE: rows x S fp16 levels -- for every group of 2^bits
+//            slots (32 * 2^bits columns) its 2^bits levels
+//            fp16(C0 + sum_i C_i b_i), entry g * 2^bits + q
 //   row_ptr  int32 [rows+1]
 //   csr      uint32 [nnz]   one outlier per word: column index in bits 0..15
 //                           (cols <= 65535), fp16 value in bits 16..31
@@ -14,6 +17,7 @@
 // 32 codes in `bits` u32 code words.  Within a record, per mode:
 //
 //   LUT_ROW, 3 bit:    3 planes of S words: word p of slot s at [p*S + s]
+//   BITPLANE, 2/3 bit: 2/3 planes of S words, as LUT_ROW 3 bit
 //   LUT_ROW, 4 bit:    S uint4 (4 code words) at [4s .. 4s+3]
 //   AFFINE_G16, 3 bit: groups of 32 slots, 136 words apart: group g holds
 //                      the zero bytes of its slots (8 words; byte t =
@@ -31,6 +35,7 @@
 // their slot at +32 + 16*lane.)
 //
 // Code bits inside a slot.  4-bit: column c in word c/8, bits 4(c%8)..+3.
+// 2-bit: column c in word c/16, bits 2(c%16)..+1.
 // 3-bit: word w (0..2) holds columns 10w..10w+9 as five adjacent pairs; pair
 // j (columns 10w+2j, 10w+2j+1) sits at half-word bit h_j of the low half
 // (even column) and of the high half (odd column), h = 0, 3, 6, 10, 13.  One
@@ -76,7 +81,7 @@ constexpr int kAff3GroupWords = 136;  // 8 words of zero bytes + 32 slot uint4
 
 __host__ __device__ inline int row_words_of(int bits, int mode, int S) {
     int w;
-    if (mode == 0)
+    if (mode != 1)
         w = bits * S;
     else if (bits == 3)
         w = S == 0 ? 0 : kAff3GroupWords * ((S - 1) / 32) + 8 + 4 * (S - 32 * ((S - 1) / 32));
@@ -98,6 +103,11 @@ __host__ __device__ inline void code_bit_place(int bits, int c, int k, int *word
         *pos = 4 * (c & 7) + k;
         return;
     }
+    if (bits == 2) {
+        *word = c >> 4;
+        *pos = 2 * (c & 15) + k;
+        return;
+    }
     if (c < 30) {
         const int t = c % 10, j = t >> 1;
         *word = c / 10;
@@ -110,7 +120,7 @@ __host__ __device__ inline void code_bit_place(int bits, int c, int k, int *word
 
 // Word index (inside a record) of code word p of slot s.
 __host__ __device__ inline int code_word_index(int bits, int mode, int S, int s, int p) {
-    if (bits == 3 && mode == 0) return p * S + s;
+    if ((bits == 3 && mode == 0) || mode == 2) return p * S + s;
     if (bits == 3) return kAff3GroupWords * (s / 32) + 8 + 4 * (s % 32) + p;
     return 4 * s + p;
 }

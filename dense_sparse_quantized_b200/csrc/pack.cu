@@ -5,6 +5,8 @@
 
 #include <vector>
 
+#include <cuda_fp16.h>
+
 #include "../../include/dsq.h"
 #include "layout.h"
 #include "internal.h"
@@ -25,8 +27,14 @@ static inline uint64_t align_up(uint64_t v, uint64_t a) { return (v + a - 1) / a
 int check_desc(const dsq_desc *d) {
     if (!d) return DSQ_ERR_INVALID_ARG;
     if (d->rows < 0 || d->cols < 0 || d->cols % kGroup != 0) return DSQ_ERR_INVALID_ARG;
-    if (d->bits != 3 && d->bits != 4) return DSQ_ERR_INVALID_ARG;
-    if (d->mode != DSQ_MODE_LUT_ROW && d->mode != DSQ_MODE_AFFINE_G16) return DSQ_ERR_INVALID_ARG;
+    if (d->mode != DSQ_MODE_LUT_ROW && d->mode != DSQ_MODE_AFFINE_G16 && d->mode != DSQ_MODE_BITPLANE)
+        return DSQ_ERR_INVALID_ARG;
+    if (d->mode == DSQ_MODE_BITPLANE) {
+        if (d->bits != 2 && d->bits != 3) return DSQ_ERR_INVALID_ARG;
+        if (d->cols % (32 << d->bits) != 0) return DSQ_ERR_INVALID_ARG;
+    } else if (d->bits != 3 && d->bits != 4) {
+        return DSQ_ERR_INVALID_ARG;
+    }
     if (d->nnz < 0 || d->nnz > (int64_t)d->rows * d->cols) return DSQ_ERR_INVALID_ARG;
     if (d->cols > 65535) return DSQ_ERR_UNSUPPORTED;
     return DSQ_OK;
@@ -50,6 +58,8 @@ void plan_blob(const dsq_desc *d, BlobHeader *h) {
     h->off_table = off;
     if (d->mode == DSQ_MODE_LUT_ROW)
         off = align_up(off + (uint64_t)d->rows * (1u << d->bits) * 2, kSectionAlign);
+    else if (d->mode == DSQ_MODE_BITPLANE)
+        off = align_up(off + (uint64_t)d->rows * h->slots * 2, kSectionAlign);
     h->off_row_ptr = off;
     off = align_up(off + (uint64_t)(d->rows + 1) * 4, kSectionAlign);
     h->off_csr = off;
@@ -121,10 +131,11 @@ extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t 
     const int64_t M = d->rows, N = d->cols, nnz = d->nnz;
     const int bits = d->bits, mode = d->mode, K = 1 << bits, qmax = K - 1;
     const int64_t G = N / kGroup;
+    const int64_t GB = mode == DSQ_MODE_BITPLANE ? N / (32 << bits) : 0;  // bit-plane groups per row
     const bool any = M * N > 0;
     if (any && !codes) return DSQ_ERR_INVALID_ARG;
     if (M > 0 && (mode == DSQ_MODE_LUT_ROW || G > 0) && !table) return DSQ_ERR_INVALID_ARG;
-    if (mode == DSQ_MODE_LUT_ROW && zeros) return DSQ_ERR_INVALID_ARG;
+    if (mode != DSQ_MODE_AFFINE_G16 && zeros) return DSQ_ERR_INVALID_ARG;
     if (mode == DSQ_MODE_AFFINE_G16 && any && !zeros) return DSQ_ERR_INVALID_ARG;
     if (M > 0 && !row_ptr) return DSQ_ERR_INVALID_ARG;
     if (nnz > 0 && (!col_idx || !values)) return DSQ_ERR_INVALID_ARG;
@@ -132,9 +143,27 @@ extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t 
     // ---- validate every input before writing anything
     for (int64_t t = 0; t < M * N; t++)
         if (codes[t] > qmax) return DSQ_ERR_INVALID_ARG;
+    std::vector<uint16_t> levels;  // BITPLANE: rows x GB x K level table
     if (mode == DSQ_MODE_LUT_ROW) {
         for (int64_t t = 0; t < M * K; t++)
             if (!isfinite(half_bits_to_double(table[t]))) return DSQ_ERR_INVALID_ARG;
+    } else if (mode == DSQ_MODE_BITPLANE) {
+        levels.resize((size_t)(M * GB * K));
+        for (int64_t t = 0; t < M * GB; t++) {
+            double c[4];
+            for (int i = 0; i <= bits; i++) {
+                c[i] = half_bits_to_double(table[t * (bits + 1) + i]);
+                if (!isfinite(c[i])) return DSQ_ERR_INVALID_ARG;
+            }
+            for (int q = 0; q < K; q++) {
+                double w = c[0];  // fp16 terms: the sum is exact in fp64
+                for (int i = 1; i <= bits; i++)
+                    if ((q >> (i - 1)) & 1) w += c[i];
+                const uint16_t hb = __half_as_ushort(__double2half(w));  // one round-to-nearest-even
+                if ((hb & 0x7C00u) == 0x7C00u) return DSQ_ERR_INVALID_ARG;
+                levels[(size_t)(t * K + q)] = hb;
+            }
+        }
     } else {
         for (int64_t t = 0; t < M * G; t++) {
             double s = half_bits_to_double(table[t]);
@@ -201,6 +230,7 @@ extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t 
         }
     }
     if (mode == DSQ_MODE_LUT_ROW && M > 0) memcpy(blob + h.off_table, table, (size_t)M * K * 2);
+    if (mode == DSQ_MODE_BITPLANE && M > 0) memcpy(blob + h.off_table, levels.data(), levels.size() * 2);
     if (M > 0) memcpy(blob + h.off_row_ptr, row_ptr, (size_t)(M + 1) * 4);
     else memset(blob + h.off_row_ptr, 0, 4);
     uint32_t *csr = (uint32_t *)(blob + h.off_csr);

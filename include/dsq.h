@@ -14,7 +14,12 @@
  *                          an fp16 scale and an integral fp16 zero per group
  *                          of 16 inputs (SpQR page, quant_config "wbits",
  *                          "groupsize": 16; the formula is this library's
- *                          reading, the page prints none).
+ *                          reading, the page prints none), or
+ *   - DSQ_MODE_BITPLANE:   w = fp16(C0 + sum_{i=1..k} C_i * b_i), k = bits
+ *                          bit planes b_i = bit (i-1) of q and k+1 fp16
+ *                          coefficients per group of 32 * 2^k inputs
+ *                          (BPDQ page, "1. Formulation de la Grille
+ *                          Variable"); the sum is exact, rounded once.
  * At the positions of the outliers the dense part holds "holes" whose codes
  * still decode (to 0 when the encoder chose q = zero).
  * W_sparse holds the outliers as fp16 CSR: values / col_idx / row_ptr (SpQR
@@ -60,12 +65,14 @@ typedef enum {
     DSQ_ERR_SCRATCH_LIMIT = -7    /* dsq_gemv_noalloc: the problem needs more than its fixed scratch */
 } dsq_status;
 
-enum { DSQ_MODE_LUT_ROW = 0, DSQ_MODE_AFFINE_G16 = 1 };
+enum { DSQ_MODE_LUT_ROW = 0, DSQ_MODE_AFFINE_G16 = 1, DSQ_MODE_BITPLANE = 2 };
 
 /* Shape and encoding of one quantized weight matrix (rows = out features M,
  * cols = in features N).  Requirements: rows >= 0; cols >= 0 and
  * cols % 16 == 0; cols <= 65535 (column indices are stored in 16 bits);
- * bits in {3, 4}; mode one of DSQ_MODE_*; 0 <= nnz <= rows*cols. */
+ * bits in {3, 4} for DSQ_MODE_LUT_ROW and DSQ_MODE_AFFINE_G16, in {2, 3}
+ * for DSQ_MODE_BITPLANE (there also cols % (32 << bits) == 0);
+ * 0 <= nnz <= rows*cols. */
 typedef struct {
     int32_t rows;
     int32_t cols;
@@ -83,9 +90,11 @@ typedef struct dsq_handle_s *dsq_handle_t;
  *   d        host; shape and encoding.
  *   codes    host uint8 [rows][cols] row-major, one code per byte, < 2^bits.
  *   table    host fp16.  LUT_ROW: [rows][2^bits] centroids.  AFFINE_G16:
- *            [rows][cols/16] scales.  All finite.
+ *            [rows][cols/16] scales.  BITPLANE: [rows][cols/(32<<bits)]
+ *            [bits+1] coefficients C0..Ck of each group; every level
+ *            C0 + sum_i C_i b_i must round to a finite fp16.  All finite.
  *   zeros    host fp16 [rows][cols/16] (AFFINE_G16: integral values in
- *            [0, 2^bits-1]); must be NULL for LUT_ROW.  For AFFINE_G16,
+ *            [0, 2^bits-1]); must be NULL for LUT_ROW and BITPLANE.  For AFFINE_G16,
  *            |scale| * max(zero, 2^bits-1-zero) must stay below 65520 so
  *            every decoded weight is finite.
  *   row_ptr  host int32 [rows+1]: row_ptr[0] = 0, nondecreasing,
@@ -137,7 +146,8 @@ DSQ_API int dsq_create(const void *packed, size_t bytes, int device, dsq_handle_
  *          element written once, rounded to nearest from an fp32 sum.
  *   batch  >= 1.  Affine 3-bit matrices take the tensor-core path from 3
  *          rows on (from 16 when a row holds more than 256 outliers);
- *          table matrices take a CUDA-core kernel, 4 rows per launch;
+ *          table and bit-plane matrices take a CUDA-core kernel, 4 rows
+ *          per launch;
  *          affine 4-bit matrices take the one-warp-per-row kernel.
  *   stream cudaStream_t of the handle's device, as void*.
  * x and y are the caller's and must not overlap.  The handle is read-only

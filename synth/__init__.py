@@ -38,7 +38,13 @@ import numpy as np
 
 LUT = "lut"
 AFFINE = "affine"
+BITPLANE = "bitplane"
 GROUP = 16
+
+
+def bitplane_group(bits: int) -> int:
+    """Inputs per coefficient group of a bit-plane matrix with `bits` planes."""
+    return 32 << bits
 
 
 def round_half_up(v: float) -> int:
@@ -95,6 +101,8 @@ class Problem:
         codes = self.rows * self.cols * self.bits // 8
         if self.mode == LUT:
             meta = self.rows * (1 << self.bits) * 2
+        elif self.mode == BITPLANE:
+            meta = self.rows * (self.cols // bitplane_group(self.bits)) * (self.bits + 1) * 2
         else:
             meta = self.rows * (self.cols // GROUP) * 4
         csr = self.nnz * 6 + (self.rows + 1) * 4
@@ -226,6 +234,31 @@ def _quantize_affine(Wd: np.ndarray, bits: int):
     return codes, s16, f16_bits(zero)
 
 
+def _quantize_bitplane(Wd: np.ndarray, hole: np.ndarray, bits: int):
+    """Bit planes and per-group coefficients (BPDQ page, "Optimisation":
+    planes from a bit-plane decomposition, coefficients by least squares).
+    Without a Hessian the metric is the identity: each group's non-hole
+    weights are rounded onto a uniform k-bit grid spanning their range (0
+    included), the planes are that code's bits, and C0..Ck are the least-
+    squares fit of the weights on [1, b_1, .., b_k], rounded to fp16."""
+    M, N = Wd.shape
+    K, G = 1 << bits, bitplane_group(bits)
+    ng = N // G
+    W3 = np.where(hole, 0.0, Wd).reshape(M, ng, G)
+    keep = (~hole).reshape(M, ng, G)
+    mn = np.minimum(np.where(keep, W3, np.inf).min(axis=2), 0.0)
+    mx = np.maximum(np.where(keep, W3, -np.inf).max(axis=2), 0.0)
+    step = (mx - mn) / (K - 1)
+    step = np.where(step > 0, step, 1.0)
+    q = np.clip(np.rint((W3 - mn[:, :, None]) / step[:, :, None]), 0, K - 1).astype(np.int64)
+    planes = np.stack([(q >> i) & 1 for i in range(bits)], axis=3).astype(np.float64)  # M, ng, G, k
+    A = np.concatenate([np.ones((M, ng, G, 1)), planes], axis=3) * keep[:, :, :, None]
+    AtA = np.einsum("mgjp,mgjq->mgpq", A, A)
+    Atw = np.einsum("mgjp,mgj->mgp", A, W3 * keep)
+    coef = np.einsum("mgpq,mgq->mgp", np.linalg.pinv(AtA), Atw)
+    return q.reshape(M, N).astype(np.uint8), f16_bits(coef)
+
+
 # ---------------------------------------------------------------- assembly
 
 def make_problem(rows: int, cols: int, bits: int, mode: str, density: float,
@@ -273,6 +306,11 @@ def make_problem(rows: int, cols: int, bits: int, mode: str, density: float,
         zeros = None
     elif mode == AFFINE:
         codes, table, zeros = _quantize_affine(Wd, bits)
+    elif mode == BITPLANE:
+        if cols % bitplane_group(bits):
+            raise ValueError("bit-plane cols must be a multiple of 32 * 2^bits")
+        codes, table = _quantize_bitplane(Wd, hole, bits)
+        zeros = None
     else:
         raise ValueError(mode)
     x = f16_bits(rng.normal(0.0, 1.0, size=(batch, N)))
@@ -300,6 +338,13 @@ CONFIGS: Dict[str, dict] = {
     "c3": dict(rows=4096, cols=11008, bits=4, mode=LUT, density=0.005,
                outliers="zipf", seed=3, batches=(1, 2, 4, 8),
                about="4096x11008 4-bit row-LUT, 0.5% Zipf(1.2) row-skewed outliers"),
+    # BPDQ variable-grid matrices on the 11008x4096 shape of c2
+    "bp2": dict(rows=11008, cols=4096, bits=2, mode=BITPLANE, density=0.01,
+                outliers="uniform", seed=52, batches=(1, 2, 4),
+                about="11008x4096 2-bit-plane BPDQ (groups of 128, 3 fp16 coefficients), 1% uniform outliers"),
+    "bp3": dict(rows=11008, cols=4096, bits=3, mode=BITPLANE, density=0.01,
+                outliers="uniform", seed=53, batches=(1, 2, 4),
+                about="11008x4096 3-bit-plane BPDQ (groups of 256, 4 fp16 coefficients), 1% uniform outliers"),
 }
 
 

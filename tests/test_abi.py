@@ -6,6 +6,7 @@ import glob
 import os
 import re
 import subprocess
+import types
 
 import numpy as np
 import pytest
@@ -170,6 +171,8 @@ def unpack_blob(blob: bytes):
     def place(c, k):
         if bits == 4:
             return c // 8, 4 * (c % 8) + k
+        if bits == 2:
+            return c // 16, 2 * (c % 16) + k
         if c < 30:
             t = c % 10
             return c // 10, (16 if t % 2 else 0) + [0, 3, 6, 10, 13][t // 2] + k
@@ -177,7 +180,7 @@ def unpack_blob(blob: bytes):
 
     def word_of(s, p_):
         # word index inside a record of code word p_ (3 = scale pair) of slot s
-        if bits == 3 and mode == 0:
+        if (bits == 3 and mode == 0) or mode == 2:
             return p_ * S + s
         if bits == 3:
             return 136 * (s // 32) + 8 + 4 * (s % 32) + p_
@@ -202,6 +205,10 @@ def unpack_blob(blob: bytes):
     if mode == 0:
         table = np.frombuffer(blob[int(off_table):int(off_table) + rows * (1 << bits) * 2],
                               np.uint16).reshape(rows, 1 << bits)
+        zeros = None
+    elif mode == 2:   # level tables: 2^bits levels of each group, rows x S
+        table = np.frombuffer(blob[int(off_table):int(off_table) + rows * S * 2],
+                              np.uint16).reshape(rows, S)
         zeros = None
     else:
         table = np.zeros((rows, G), np.uint16)
@@ -235,6 +242,57 @@ def test_layout_round_trip(bits, mode, cols):
         assert np.array_equal(zeros, p.zeros)
     assert np.array_equal(rp, p.row_ptr) and np.array_equal(ci, p.col_idx)
     assert np.array_equal(va, p.values)
+
+
+@pytest.mark.parametrize("bits,cols", [(2, 128), (2, 1024), (3, 256), (3, 4096)])
+def test_bitplane_layout_and_levels(orc, bits, cols):
+    """Bit-plane blobs: the codes round-trip, and the level table holds, for
+    every group g and code q, the oracle's decoded weight of a column of
+    group g whose code is q."""
+    p = synth.make_problem(9, cols, bits, "bitplane", 0.03, "uniform", 3 + bits, 1)
+    codes, levels, zeros, rp, ci, va = unpack_blob(dsq.pack_problem(p))
+    assert zeros is None and np.array_equal(codes, p.codes)
+    assert np.array_equal(rp, p.row_ptr) and np.array_equal(ci, p.col_idx) and np.array_equal(va, p.values)
+    K, G = 1 << bits, synth.bitplane_group(bits)
+    probe = types.SimpleNamespace(**vars(p))
+    probe.codes = np.tile(np.arange(cols) % K, (p.rows, 1)).astype(np.uint8)
+    wd = orc.decode(probe)
+    want = np.stack([wd[:, g * G:g * G + K] for g in range(cols // G)], axis=1).reshape(p.rows, -1)
+    assert np.array_equal(levels, want)
+
+
+def test_bitplane_levels_round_once(orc):
+    """Coefficients over every binade (subnormals, ties, sums past the fp16
+    range excluded): the packed levels equal the oracle's single rounding of
+    the exact sum."""
+    rng = np.random.default_rng(17)
+    for bits in (2, 3):
+        K, G = 1 << bits, synth.bitplane_group(bits)
+        rows, cols = 64, 4 * G
+        e = rng.integers(-24, 12, size=(rows, cols // G, bits + 1)).astype(np.float64)
+        v = rng.integers(1, 2048, size=e.shape) * np.exp2(e - 10) * rng.choice([-1.0, 1.0], e.shape)
+        coef = np.asarray(v, np.float64).astype(np.float16).view(np.uint16)
+        codes = np.tile(np.arange(cols) % K, (rows, 1)).astype(np.uint8)
+        p = types.SimpleNamespace(rows=rows, cols=cols, bits=bits, mode="bitplane", codes=codes,
+                                  table=coef, zeros=None, row_ptr=np.zeros(rows + 1, np.int32),
+                                  col_idx=np.zeros(0, np.int32), values=np.zeros(0, np.uint16),
+                                  x=np.zeros((1, cols), np.uint16))
+        _, levels, _, _, _, _ = unpack_blob(dsq.pack_problem(p))
+        wd = orc.decode(p)
+        want = np.stack([wd[:, g * G:g * G + K] for g in range(cols // G)], axis=1).reshape(rows, -1)
+        assert np.array_equal(levels, want), bits
+
+
+def test_bitplane_pack_rejects():
+    pb = synth.make_problem(4, 256, 2, "bitplane", 0.02, "uniform", 1, 1)
+    assert pack_status(pb) == dsq.DSQ_OK
+    assert pack_status(pb, bits=4) == dsq.DSQ_ERR_INVALID_ARG                  # 2 or 3 planes
+    assert pack_status(pb, cols=192, codes=pb.codes[:, :192]) == dsq.DSQ_ERR_INVALID_ARG  # groups of 128
+    assert pack_status(pb, zeros=np.zeros((4, 16), np.uint16)) == dsq.DSQ_ERR_INVALID_ARG
+    assert pack_status(pb, table=np.full_like(pb.table, 0x7E00)) == dsq.DSQ_ERR_INVALID_ARG   # NaN
+    big = pb.table.copy()
+    big[1, 0] = [0x7BFF, 0x7BFF, 0x0000]       # level C0 + C1 = 131008 is past fp16
+    assert pack_status(pb, table=big) == dsq.DSQ_ERR_INVALID_ARG
 
 
 def test_three_bit_fields():
@@ -277,9 +335,13 @@ def _offsets(blob: bytes):
     return rows, off_rp, off_csr
 
 
-@pytest.mark.parametrize("bits,mode", [(3, "lut"), (4, "lut"), (3, "affine"), (4, "affine")])
+@pytest.mark.parametrize("bits,mode", [(3, "lut"), (4, "lut"), (3, "affine"), (4, "affine"),
+                                       (2, "bitplane"), (3, "bitplane")])
 def test_create_accepts_packed_blobs(bits, mode):
-    for rows, cols, dens in ((7, 48, 0.05), (33, 1024, 0.02), (5, 16, 0.0), (1, 4096, 0.01)):
+    shapes = ((7, 48, 0.05), (33, 1024, 0.02), (5, 16, 0.0), (1, 4096, 0.01))
+    if mode == "bitplane":
+        shapes = ((7, 256, 0.05), (33, 1024, 0.02), (5, 256, 0.0), (1, 4096, 0.01))
+    for rows, cols, dens in shapes:
         p = synth.make_problem(rows, cols, bits, mode, dens, "uniform" if dens else "none", 9, 1)
         assert _create_rc(dsq.pack_problem(p)) in (dsq.DSQ_OK, dsq.DSQ_ERR_CUDA), (rows, cols, dens)
 

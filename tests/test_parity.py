@@ -79,9 +79,10 @@ def sample_rows(p, n=768, seed=0):
 
 SMALL_CONFIGS = ["c0", "c1", "c2", "c3"]
 C4 = ["c4_" + n for n, _, _ in synth.C4_LAYERS]
+BITPLANE = ["bp2", "bp3"]
 
 
-@pytest.mark.parametrize("name", SMALL_CONFIGS + C4)
+@pytest.mark.parametrize("name", SMALL_CONFIGS + C4 + BITPLANE)
 def test_decode_bit_exact(orc, name):
     p, h = config(name)
     got = to_bits(h.decode())
@@ -107,6 +108,35 @@ def oracle_all_rows(orc, p, x):
     with ThreadPoolExecutor(max_workers=len(slices)) as pool:
         parts = list(pool.map(lambda r: orc.gemv(p, x=x, rows=r), slices))
     return np.concatenate([a for a, _ in parts], axis=1), np.concatenate([b for _, b in parts], axis=1)
+
+
+@pytest.mark.parametrize("name", BITPLANE)
+@pytest.mark.parametrize("batch", [1, 2, 3, 4, 5])
+def test_gemv_bitplane_every_row(orc, name, batch):
+    """BPDQ matrices (11008 x 4096, 2 and 3 planes, 1% outliers): the batch-1
+    table kernel with per-group levels, the 2-4 row kernel, and both for 5
+    rows; every row against the oracle."""
+    p, h = config(name)
+    xb = synth.f16_bits(np.random.default_rng(batch).standard_normal((batch, p.cols)))
+    y = gemv(h, xb, batch)
+    y_ref, bound = oracle_all_rows(orc, p, xb)
+    check_y(y, y_ref, bound, f"{name} B={batch}")
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("rows,cols", [(1, 256), (7, 1024), (33, 4096), (130, 512), (64, 24576), (5, 25600)])
+def test_bitplane_small_shapes(orc, bits, rows, cols):
+    """Ragged row counts, one group per row up to 96 groups; 25600 columns
+    exceed the tuned kernels' 24 column warps and run the generic kernel."""
+    G = synth.bitplane_group(bits)
+    cols = max(G, cols // G * G)
+    p = synth.make_problem(rows, cols, bits, "bitplane", 0.02, "uniform", rows + bits, 3)
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        assert np.array_equal(to_bits(h.decode()), orc.decode(p))
+        for batch in (1, 2, 3):
+            y = gemv(h, p.x, batch)
+            y_ref, bound = orc.gemv(p, x=p.x[:batch])
+            check_y(y, y_ref, bound, f"{rows}x{cols} bitplane k={bits} B={batch}")
 
 
 @pytest.mark.parametrize("name", C4)
