@@ -54,6 +54,11 @@ class Oracle:
         lib.oracle_gemv_rows.restype = _I
         lib.oracle_gemv_rows.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I,
                                          _P, _P, _I, _P, _P]
+        lib.oracle_materialize_two_axis.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                                                    _P, _P, _P]
+        lib.oracle_gemv_rows_two_axis.restype = _I
+        lib.oracle_gemv_rows_two_axis.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                                                  _P, _P, _I, _P, _P, _I, _P, _P]
         self.lib = lib
         self.path = path
 
@@ -81,29 +86,34 @@ class Oracle:
         rp = np.ascontiguousarray(p.row_ptr, dtype=np.int32)
         ci = np.ascontiguousarray(p.col_idx, dtype=np.int32)
         va = np.ascontiguousarray(p.values, dtype=np.uint16)
-        keep = (codes, table, zeros, rp, ci, va)
+        rs = getattr(p, "row_scale", None)
+        cs = getattr(p, "col_scale", None)
+        rs = None if rs is None else np.ascontiguousarray(rs, dtype=np.uint16)
+        cs = None if cs is None else np.ascontiguousarray(cs, dtype=np.uint16)
+        keep = (codes, table, zeros, rp, ci, va, rs, cs)
         ptr = lambda a: None if a is None else a.ctypes.data  # noqa: E731
         return keep, (int(p.rows), int(p.cols), int(p.bits), mode, ptr(codes),
-                      ptr(table), ptr(zeros), ptr(rp), ptr(ci), ptr(va))
+                      ptr(table), ptr(zeros), ptr(rp), ptr(ci), ptr(va)), (ptr(rs), ptr(cs))
 
     def decode(self, p) -> np.ndarray:
         """W_dense as fp16 bit patterns, rows x cols."""
-        keep, a = self._args(p)
+        keep, a, _ = self._args(p)
         out = np.empty((p.rows, p.cols), dtype=np.uint16)
         self.lib.oracle_decode(*a[:7], out.ctypes.data)
         return out
 
     def materialize(self, p) -> np.ndarray:
-        """What = W_dense + W_sparse in fp64, rows x cols."""
-        keep, a = self._args(p)
+        """What = W_dense + W_sparse in fp64, rows x cols (the dense part
+        times r_i * c_j when the problem carries row_scale / col_scale)."""
+        keep, a, sc = self._args(p)
         out = np.empty((p.rows, p.cols), dtype=np.float64)
-        self.lib.oracle_materialize(*a, out.ctypes.data)
+        self.lib.oracle_materialize_two_axis(*a, *sc, out.ctypes.data)
         return out
 
     def gemv(self, p, x: Optional[np.ndarray] = None,
              rows: Optional[Sequence[int]] = None):
         """(y_ref, bound), each batch x len(rows) fp64; all rows by default."""
-        keep, a = self._args(p)
+        keep, a, sc = self._args(p)
         x = np.ascontiguousarray(p.x if x is None else x, dtype=np.uint16)
         if x.ndim == 1:
             x = x[None, :]
@@ -115,9 +125,9 @@ class Oracle:
             n = int(rl.size)
         y = np.empty((batch, n), dtype=np.float64)
         bound = np.empty((batch, n), dtype=np.float64)
-        rc = self.lib.oracle_gemv_rows(*a, batch, x.ctypes.data,
-                                       None if rl is None else rl.ctypes.data, n,
-                                       y.ctypes.data, bound.ctypes.data)
+        rc = self.lib.oracle_gemv_rows_two_axis(*a, *sc, batch, x.ctypes.data,
+                                                None if rl is None else rl.ctypes.data, n,
+                                                y.ctypes.data, bound.ctypes.data)
         if rc != 0:
             raise MemoryError("oracle_gemv_rows failed")
         return y, bound

@@ -29,6 +29,12 @@
  *    dimension.  Read as: groups of 32 * 2^k inputs, fp16 coefficients, a
  *    weight's k plane bits held in one code q with b_i = bit (i-1) of q, and
  *    the sum C_0 + sum_i C_i b_i evaluated exactly and rounded once to fp16.
+ *  - SINQ page, "Mise a l'echelle sur deux axes": a vector of scales for the
+ *    rows and another for the columns around the quantized matrix.  Read as:
+ *    the dense weight is r_i * c_j * Wd_ij with fp16 r and c and Wd the
+ *    decoded dense weight above (the product is exact in fp64 and is not
+ *    rounded); the outliers, taken from the unscaled matrix, are added
+ *    unscaled.
  *
  * Precision.  A decoded dense weight is an fp16 value: a table entry is
  * copied bit for bit; an affine weight is scale*(q-zero) evaluated exactly in
@@ -157,42 +163,72 @@ void oracle_decode(int rows, int cols, int bits, int mode, const uint8_t *codes,
                 oracle_decode_one(i, j, cols, bits, mode, codes, table, zeros);
 }
 
-/* What row i in fp64: decoded dense weights, then each CSR entry of the row
- * added to the weight at its column. */
+/* What row i in fp64: decoded dense weights (times r_i * c_j when the row
+ * and column scales are given, NULL meaning none), then each CSR entry of the
+ * row added to the weight at its column. */
+void oracle_weight_row_two_axis(int64_t i, int cols, int bits, int mode,
+                                const uint8_t *codes, const uint16_t *table,
+                                const uint16_t *zeros, const int32_t *row_ptr,
+                                const int32_t *col_idx, const uint16_t *values,
+                                const uint16_t *rscale, const uint16_t *cscale,
+                                double *wrow)
+{
+    double r = rscale ? oracle_half_to_double(rscale[i]) : 1.0;
+    for (int64_t j = 0; j < cols; j++) {
+        double c = cscale ? oracle_half_to_double(cscale[j]) : 1.0;
+        wrow[j] = r * c * oracle_half_to_double(
+            oracle_decode_one(i, j, cols, bits, mode, codes, table, zeros));
+    }
+    for (int64_t k = row_ptr[i]; k < row_ptr[i + 1]; k++)
+        wrow[col_idx[k]] += oracle_half_to_double(values[k]);
+}
+
 void oracle_weight_row(int64_t i, int cols, int bits, int mode,
                        const uint8_t *codes, const uint16_t *table,
                        const uint16_t *zeros, const int32_t *row_ptr,
                        const int32_t *col_idx, const uint16_t *values,
                        double *wrow)
 {
-    for (int64_t j = 0; j < cols; j++)
-        wrow[j] = oracle_half_to_double(
-            oracle_decode_one(i, j, cols, bits, mode, codes, table, zeros));
-    for (int64_t k = row_ptr[i]; k < row_ptr[i + 1]; k++)
-        wrow[col_idx[k]] += oracle_half_to_double(values[k]);
+    oracle_weight_row_two_axis(i, cols, bits, mode, codes, table, zeros, row_ptr,
+                               col_idx, values, NULL, NULL, wrow);
 }
 
-/* What: rows x cols fp64. */
+/* What: rows x cols fp64 (row and column scales may be NULL). */
+void oracle_materialize_two_axis(int rows, int cols, int bits, int mode,
+                                 const uint8_t *codes, const uint16_t *table,
+                                 const uint16_t *zeros, const int32_t *row_ptr,
+                                 const int32_t *col_idx, const uint16_t *values,
+                                 const uint16_t *rscale, const uint16_t *cscale,
+                                 double *w)
+{
+    for (int64_t i = 0; i < rows; i++)
+        oracle_weight_row_two_axis(i, cols, bits, mode, codes, table, zeros,
+                                   row_ptr, col_idx, values, rscale, cscale,
+                                   w + i * cols);
+}
+
 void oracle_materialize(int rows, int cols, int bits, int mode,
                         const uint8_t *codes, const uint16_t *table,
                         const uint16_t *zeros, const int32_t *row_ptr,
                         const int32_t *col_idx, const uint16_t *values,
                         double *w)
 {
-    for (int64_t i = 0; i < rows; i++)
-        oracle_weight_row(i, cols, bits, mode, codes, table, zeros, row_ptr,
-                          col_idx, values, w + i * cols);
+    oracle_materialize_two_axis(rows, cols, bits, mode, codes, table, zeros,
+                                row_ptr, col_idx, values, NULL, NULL, w);
 }
 
 /* y_ref and bound for the listed output rows only (all rows when
  * row_list == NULL, n_list == rows).  x: batch x cols fp16; y_ref and bound:
- * batch x n_list fp64, column t holding row row_list[t]. */
-int oracle_gemv_rows(int rows, int cols, int bits, int mode,
-                     const uint8_t *codes, const uint16_t *table,
-                     const uint16_t *zeros, const int32_t *row_ptr,
-                     const int32_t *col_idx, const uint16_t *values, int batch,
-                     const uint16_t *x, const int32_t *row_list, int n_list,
-                     double *y_ref, double *bound)
+ * batch x n_list fp64, column t holding row row_list[t].  Row and column
+ * scales may be NULL. */
+int oracle_gemv_rows_two_axis(int rows, int cols, int bits, int mode,
+                              const uint8_t *codes, const uint16_t *table,
+                              const uint16_t *zeros, const int32_t *row_ptr,
+                              const int32_t *col_idx, const uint16_t *values,
+                              const uint16_t *rscale, const uint16_t *cscale,
+                              int batch, const uint16_t *x,
+                              const int32_t *row_list, int n_list,
+                              double *y_ref, double *bound)
 {
     double *wrow = (double *)malloc(sizeof(double) * (cols > 0 ? cols : 1));
     double *xd = (double *)malloc(sizeof(double) * ((int64_t)batch * cols + 1));
@@ -205,8 +241,9 @@ int oracle_gemv_rows(int rows, int cols, int bits, int mode,
         xd[t] = oracle_half_to_double(x[t]);
     for (int t = 0; t < n_list; t++) {
         int64_t i = row_list ? row_list[t] : t;
-        oracle_weight_row(i, cols, bits, mode, codes, table, zeros, row_ptr,
-                          col_idx, values, wrow);
+        oracle_weight_row_two_axis(i, cols, bits, mode, codes, table, zeros,
+                                   row_ptr, col_idx, values, rscale, cscale,
+                                   wrow);
         for (int b = 0; b < batch; b++) {
             double acc = 0.0, mag = 0.0;
             for (int64_t j = 0; j < cols; j++) {
@@ -221,6 +258,19 @@ int oracle_gemv_rows(int rows, int cols, int bits, int mode,
     free(wrow);
     free(xd);
     return 0;
+}
+
+int oracle_gemv_rows(int rows, int cols, int bits, int mode,
+                     const uint8_t *codes, const uint16_t *table,
+                     const uint16_t *zeros, const int32_t *row_ptr,
+                     const int32_t *col_idx, const uint16_t *values, int batch,
+                     const uint16_t *x, const int32_t *row_list, int n_list,
+                     double *y_ref, double *bound)
+{
+    return oracle_gemv_rows_two_axis(rows, cols, bits, mode, codes, table,
+                                     zeros, row_ptr, col_idx, values, NULL,
+                                     NULL, batch, x, row_list, n_list, y_ref,
+                                     bound);
 }
 
 /* Full product: y_ref, bound are batch x rows. */

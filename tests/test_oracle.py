@@ -231,6 +231,35 @@ def pin_bitplane_uniform_grid_is_affine(orc):
             assert np.array_equal(orc.decode(bp), orc.decode(af)), (k, s, z)
 
 
+def pin_two_axis_golden(orc):
+    """The hand-worked two-axis example (SINQ page, "Mise a l'echelle sur deux
+    axes"): What = r_i c_j Wd_ij plus the unscaled outliers, and its product."""
+    g = json.load(open(os.path.join(GOLDEN, "two_axis_example.json")))
+    h = lambda v: [int(t, 16) for t in v]  # noqa: E731
+    p = problem(g["rows"], g["cols"], g["bits"], "lut", np.array(g["codes"]).reshape(-1),
+                [h(r) for r in g["table"]], None, g["row_ptr"], g["col_idx"], h(g["values"]), h(g["x"]))
+    p.row_scale = np.array(h(g["row_scale"]), np.uint16)
+    p.col_scale = np.array(h(g["col_scale"]), np.uint16)
+    assert np.array_equal(orc.materialize(p), np.array(g["what"]))
+    y, bd = orc.gemv(p)
+    assert np.array_equal(y[0], np.array(g["y"])) and np.array_equal(bd[0], np.array(g["bound"]))
+
+
+def pin_two_axis_unit_scales(orc):
+    """All-one row and column scales leave every result of the plain product
+    unchanged, bit for bit (every mode)."""
+    rng = np.random.default_rng(31)
+    for bits, mode, cols in ((3, "lut", 48), (4, "affine", 64), (2, "bitplane", 256)):
+        p = random_problem(rng, 6, cols, bits, mode, 2)
+        y0, b0 = orc.gemv(p)
+        w0 = orc.materialize(p)
+        p.row_scale = np.full(p.rows, 0x3C00, np.uint16)
+        p.col_scale = np.full(p.cols, 0x3C00, np.uint16)
+        y1, b1 = orc.gemv(p)
+        assert np.array_equal(y0, y1) and np.array_equal(b0, b1)
+        assert np.array_equal(w0, orc.materialize(p))
+
+
 # ------------------------------------------------------------------ product pins
 
 def exact_reference(p):
@@ -338,6 +367,7 @@ def pin_rows_subset(orc):
 PINS = [pin_half_to_double_exhaustive, pin_double_to_half, pin_csr_example,
         pin_lut_decode_identity, pin_affine_decode_golden, pin_affine_group_layout,
         pin_bitplane_decode_golden, pin_bitplane_group_layout, pin_bitplane_uniform_grid_is_affine,
+        pin_two_axis_golden, pin_two_axis_unit_scales,
         pin_gemv_exact, pin_special_cases, pin_decomposition, pin_rows_subset]
 
 
@@ -378,6 +408,11 @@ MUTANTS = {
                                  "                w = oracle_half_to_double(oracle_double_to_half(w + oracle_half_to_double(c[p])));"),
     "bitplane_coef_row_stride": ("table + (i * (cols / gsize) + j / gsize) * (bits + 1)",
                                  "table + (j / gsize) * (bits + 1)"),
+    "two_axis_scaled_outliers": ("        wrow[col_idx[k]] += oracle_half_to_double(values[k]);\n}\n\nvoid oracle_weight_row(",
+                                 "        wrow[col_idx[k]] += r * oracle_half_to_double(values[k]);\n}\n\nvoid oracle_weight_row("),
+    "two_axis_col_by_row": ("double c = cscale ? oracle_half_to_double(cscale[j]) : 1.0;",
+                            "double c = cscale ? oracle_half_to_double(cscale[i]) : 1.0;"),
+    "two_axis_no_row_scale": ("double r = rscale ? oracle_half_to_double(rscale[i]) : 1.0;", "double r = 1.0;"),
     "first_column_skipped": ("for (int64_t j = 0; j < cols; j++) {\n                acc",
                              "for (int64_t j = 1; j < cols; j++) {\n                acc"),
 }
