@@ -32,7 +32,7 @@ MODE_LUT_ROW = 0
 MODE_AFFINE_G16 = 1
 MODE_BITPLANE = 2
 
-EXPORTS = ("dsq_pack", "dsq_blob_desc", "dsq_create", "dsq_gemv", "dsq_gemv_launches", "dsq_decode",
+EXPORTS = ("dsq_pack", "dsq_pack_two_axis", "dsq_blob_desc", "dsq_create", "dsq_gemv", "dsq_gemv_launches", "dsq_decode",
            "dsq_handle_desc", "dsq_device_bytes", "dsq_check", "dsq_destroy", "dsq_status_string",
            "dsq_gemv_noalloc", "dsq_selftest_wait_timeout")
 
@@ -61,6 +61,8 @@ def library() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIBRARY)
         P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         lib.dsq_pack.argtypes = [ctypes.POINTER(Desc), P, P, P, P, P, P, P, ctypes.POINTER(SZ)]
+        lib.dsq_pack_two_axis.argtypes = [ctypes.POINTER(Desc), P, P, P, P, P, P, P, P, P,
+                                          ctypes.POINTER(SZ)]
         lib.dsq_blob_desc.argtypes = [P, SZ, ctypes.POINTER(Desc)]
         lib.dsq_create.argtypes = [P, SZ, I, ctypes.POINTER(P)]
         lib.dsq_gemv.argtypes = [P, P, P, I, P]
@@ -99,27 +101,32 @@ def _arr(a, dtype):
 
 
 def pack(rows: int, cols: int, bits: int, mode, codes, table, zeros, row_ptr, col_idx,
-         values) -> bytes:
+         values, row_scale=None, col_scale=None) -> bytes:
     """Validate logical weights and return the packed blob (host bytes).
 
     mode: 'lut' / 'affine' / 'bitplane' or MODE_*.  Arrays: codes uint8
     [rows, cols]; table fp16 bits (uint16) [rows, 2^bits] (lut),
     [rows, cols/16] (affine scales) or [rows, cols/(32*2^bits), bits+1]
     (bit-plane coefficients C0..Ck); zeros uint16 [rows, cols/16] or None;
-    row_ptr int32; col_idx int32; values uint16 fp16 bits."""
+    row_ptr int32; col_idx int32; values uint16 fp16 bits.  row_scale /
+    col_scale (fp16 bits [rows] / [cols]): two-axis scales (dsq_pack_two_axis)."""
     lib = library()
     m = {"lut": MODE_LUT_ROW, "affine": MODE_AFFINE_G16, "bitplane": MODE_BITPLANE}.get(mode, mode)
     nnz = int(np.asarray(row_ptr)[-1]) if row_ptr is not None and len(row_ptr) else 0
     d = Desc(int(rows), int(cols), int(bits), int(m), nnz)
     keep = [_arr(codes, np.uint8), _arr(table, np.uint16), _arr(zeros, np.uint16),
             _arr(row_ptr, np.int32), _arr(col_idx, np.int32), _arr(values, np.uint16)]
+    two = row_scale is not None or col_scale is not None
+    if two:
+        keep += [_arr(row_scale, np.uint16), _arr(col_scale, np.uint16)]
     ptrs = [p for _, p in keep]
+    fn, name = (lib.dsq_pack_two_axis, "dsq_pack_two_axis") if two else (lib.dsq_pack, "dsq_pack")
     size = ctypes.c_size_t(0)
-    rc = lib.dsq_pack(ctypes.byref(d), *ptrs, None, ctypes.byref(size))
+    rc = fn(ctypes.byref(d), *ptrs, None, ctypes.byref(size))
     if rc != DSQ_ERR_BUFFER_TOO_SMALL:
-        _check(rc, "dsq_pack")
+        _check(rc, name)
     buf = ctypes.create_string_buffer(size.value)
-    _check(lib.dsq_pack(ctypes.byref(d), *ptrs, buf, ctypes.byref(size)), "dsq_pack")
+    _check(fn(ctypes.byref(d), *ptrs, buf, ctypes.byref(size)), name)
     return buf.raw[:size.value]
 
 
@@ -127,7 +134,7 @@ def pack_problem(p) -> bytes:
     """pack() from an object with rows, cols, bits, mode, codes, table, zeros,
     row_ptr, col_idx, values attributes."""
     return pack(p.rows, p.cols, p.bits, p.mode, p.codes, p.table, p.zeros, p.row_ptr,
-                p.col_idx, p.values)
+                p.col_idx, p.values, getattr(p, "row_scale", None), getattr(p, "col_scale", None))
 
 
 def blob_desc(blob: bytes) -> Desc:

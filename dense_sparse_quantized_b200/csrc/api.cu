@@ -92,6 +92,10 @@ extern "C" int dsq_create(const void *packed, size_t bytes, int device, dsq_hand
     m.table = (const uint16_t *)(h->d_blob + hd.off_table);
     m.row_ptr = (const int32_t *)(h->d_blob + hd.off_row_ptr);
     m.csr = (const uint32_t *)(h->d_blob + hd.off_csr);
+    if (hd.flags & kFlagTwoAxis) {
+        m.rscale = (const uint16_t *)(h->d_blob + hd.off_rscale);
+        m.cscale = (const uint16_t *)(h->d_blob + hd.off_cscale);
+    }
     if (cudaMalloc(&h->d_status, sizeof(int)) != cudaSuccess) {
         cudaGetLastError();
         dsq_destroy(h);

@@ -172,8 +172,9 @@ __device__ __forceinline__ void reduce_pieces(const TileDesc &td, unsigned char 
     }
 }
 
-// y[r] = fp16(dense_scale * sum_c part[i][c] + sum of the row's piece sums),
-// in a fixed order per row.  Warp w takes rows 32w + lane, 32w + lane + 32W,
+// y[r] = fp16(dense_scale * r_i * sum_c part[i][c] + sum of the row's piece
+// sums), in a fixed order per row (r_i = the row scale of a two-axis matrix,
+// else 1).  Warp w takes rows 32w + lane, 32w + lane + 32W,
 // ...: a lane sums the pieces of a row with <= kHeavyPieces of them, the
 // whole warp those of a longer row.
 __device__ __forceinline__ void finalize(const TileDesc &td, const unsigned char *smem, const B1Params &p,
@@ -208,7 +209,8 @@ __device__ __forceinline__ void finalize(const TileDesc &td, const unsigned char
         if (i < nrows) {
             float acc = 0.f;
             for (int c = 0; c < p.C; c++) acc += part[(size_t)i * p.C + c];
-            y[td.r0 + i] = __float2half_rn(fmaf(acc, dense_scale, o));
+            const float rs = p.m.rscale ? __half2float(__ushort_as_half(p.m.rscale[td.r0 + i])) : 1.0f;
+            y[td.r0 + i] = __float2half_rn(fmaf(acc, dense_scale * rs, o));
         }
     }
 }
@@ -575,6 +577,18 @@ b1_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y) 
                 xr[2 * i] = f.x;
                 xr[2 * i + 1] = f.y;
             }
+            if (m.cscale) {
+                // two-axis: the dense part sees c_j x_j, exact in fp32; the
+                // outliers keep the staged, unscaled x
+                uint32_t ch[16];
+                x_pairs(reinterpret_cast<const __half *>(m.cscale), s, m.cols, ch);
+#pragma unroll
+                for (int i = 0; i < 16; i++) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ch[i]));
+                    xr[2 * i] *= f.x;
+                    xr[2 * i + 1] *= f.y;
+                }
+            }
             if (rg == 0) stage_x(smem, p, s, xh);
         }
         float *part = reinterpret_cast<float *>(smem + p.off_part);
@@ -810,7 +824,8 @@ enum Kind { kNone = -1, kAff3 = 0, kLut3 = 3, kLut4 = 4, kBp2 = 12, kBp3 = 13 };
 Kind b1_kind(const MatrixView &m, int batch) {
     if (batch != 1 || m.rows <= 0 || m.cols <= 0) return kNone;
     if ((m.slots + 31) / 32 > kMaxWarps) return kNone;
-    if (m.mode == DSQ_MODE_AFFINE_G16) return m.bits == 3 ? kAff3 : kNone;
+    // the affine kernel multiplies fp16 x, which cannot hold c_j x_j exactly
+    if (m.mode == DSQ_MODE_AFFINE_G16) return m.bits == 3 && !m.cscale ? kAff3 : kNone;
     if (m.mode == DSQ_MODE_BITPLANE) return m.bits == 2 ? kBp2 : kBp3;
     return m.bits == 3 ? kLut3 : kLut4;
 }
@@ -1018,7 +1033,7 @@ int batched_launch_count(const dsq_handle_s *h, int batch) {
     B1Params p;
     size_t smem;
     const MatrixView &m = h->view;
-    if (batch < 2 || m.mode == DSQ_MODE_AFFINE_G16 || m.rows <= 0 || m.cols <= 0 || h->sched.n_tiles == 0 ||
+    if (batch < 2 || m.mode == DSQ_MODE_AFFINE_G16 || m.cscale || m.rows <= 0 || m.cols <= 0 || h->sched.n_tiles == 0 ||
         !plan_bn(h, 4, &p, &smem))
         return -1;
     return (batch + 3) / 4;

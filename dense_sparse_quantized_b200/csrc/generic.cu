@@ -56,7 +56,10 @@ __device__ __forceinline__ const __half *row_table_of(const MatrixView &m, int r
     return nullptr;
 }
 
-template <int BITS, int MODE, int BC>
+// TWO: two-axis scales -- the dense weights multiply c_j x_j (exact in fp32)
+// and the row's dense sum is multiplied by r_i before the outliers, which use
+// the unscaled x, are added.
+template <int BITS, int MODE, int BC, bool TWO>
 __global__ void __launch_bounds__(256) gemv_generic_kernel(MatrixView m, const __half *__restrict__ x,
                                                            __half *__restrict__ y, int batch, int b0) {
     const int lane = threadIdx.x & 31;
@@ -66,9 +69,9 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(MatrixView m, const _
     const int N = m.cols;
     const uint32_t *rec = m.dense + (size_t)row * m.row_words;
     const __half *row_table = row_table_of<BITS, MODE>(m, row);
-    float acc[BC];
+    float acc[BC], aco[BC];  // dense and (two-axis only) outlier sums
 #pragma unroll
-    for (int b = 0; b < BC; b++) acc[b] = 0.f;
+    for (int b = 0; b < BC; b++) acc[b] = aco[b] = 0.f;
 
     for (int s = lane; s < m.slots; s += 32) {
         uint32_t w[4] = {0, 0, 0, 0}, scales = 0, zb = 0;
@@ -78,9 +81,10 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(MatrixView m, const _
             const int j = s * 32 + c;
             if (j < N) {
                 float wv = __half2float(decode_weight<BITS, MODE>(row_table, slot_code<BITS>(w, c), scales, zb, c, s));
+                const float cj = TWO ? __half2float(__ushort_as_half(m.cscale[j])) : 1.0f;
 #pragma unroll
                 for (int b = 0; b < BC; b++)
-                    if (b < nb) acc[b] = fmaf(wv, __half2float(x[(size_t)(b0 + b) * N + j]), acc[b]);
+                    if (b < nb) acc[b] = fmaf(wv, __half2float(x[(size_t)(b0 + b) * N + j]) * cj, acc[b]);
             }
         }
     }
@@ -91,14 +95,21 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(MatrixView m, const _
         const int j = (int)(e & 0xffffu);
 #pragma unroll
         for (int b = 0; b < BC; b++)
-            if (b < nb) acc[b] = fmaf(v, __half2float(x[(size_t)(b0 + b) * N + j]), acc[b]);
+            if (b < nb) {
+                if (TWO) aco[b] = fmaf(v, __half2float(x[(size_t)(b0 + b) * N + j]), aco[b]);
+                else acc[b] = fmaf(v, __half2float(x[(size_t)(b0 + b) * N + j]), acc[b]);
+            }
     }
+    const float rs = TWO ? __half2float(__ushort_as_half(m.rscale[row])) : 1.0f;
 #pragma unroll
     for (int b = 0; b < BC; b++) {
-        float a = acc[b];
+        float a = acc[b], o = aco[b];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == 0 && b < nb) y[(size_t)(b0 + b) * m.rows + row] = __float2half_rn(a);
+        for (int d = 16; d > 0; d >>= 1) {
+            a += __shfl_xor_sync(0xffffffffu, a, d);
+            if (TWO) o += __shfl_xor_sync(0xffffffffu, o, d);
+        }
+        if (lane == 0 && b < nb) y[(size_t)(b0 + b) * m.rows + row] = __float2half_rn(TWO ? fmaf(a, rs, o) : a);
     }
 }
 
@@ -124,19 +135,25 @@ __global__ void zero_kernel(__half *y, int64_t n) {
         y[i] = __ushort_as_half(0);
 }
 
-template <int BITS, int MODE>
-static void launch_generic_t(const MatrixView &m, const __half *x, __half *y, int batch, cudaStream_t st) {
+template <int BITS, int MODE, bool TWO>
+static void launch_generic_tt(const MatrixView &m, const __half *x, __half *y, int batch, cudaStream_t st) {
     const int warps = 8;
     dim3 grid((m.rows + warps - 1) / warps);
     for (int b0 = 0; b0 < batch; b0 += 8) {
         int nb = batch - b0;
         if (nb == 1)
-            gemv_generic_kernel<BITS, MODE, 1><<<grid, warps * 32, 0, st>>>(m, x, y, batch, b0);
+            gemv_generic_kernel<BITS, MODE, 1, TWO><<<grid, warps * 32, 0, st>>>(m, x, y, batch, b0);
         else if (nb <= 4)
-            gemv_generic_kernel<BITS, MODE, 4><<<grid, warps * 32, 0, st>>>(m, x, y, batch, b0);
+            gemv_generic_kernel<BITS, MODE, 4, TWO><<<grid, warps * 32, 0, st>>>(m, x, y, batch, b0);
         else
-            gemv_generic_kernel<BITS, MODE, 8><<<grid, warps * 32, 0, st>>>(m, x, y, batch, b0);
+            gemv_generic_kernel<BITS, MODE, 8, TWO><<<grid, warps * 32, 0, st>>>(m, x, y, batch, b0);
     }
+}
+
+template <int BITS, int MODE>
+static void launch_generic_t(const MatrixView &m, const __half *x, __half *y, int batch, cudaStream_t st) {
+    if (m.cscale) launch_generic_tt<BITS, MODE, true>(m, x, y, batch, st);
+    else launch_generic_tt<BITS, MODE, false>(m, x, y, batch, st);
 }
 
 int launch_gemv_generic(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t st) {

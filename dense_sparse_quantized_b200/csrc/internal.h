@@ -13,7 +13,7 @@ namespace dsq {
 
 double half_bits_to_double(uint16_t h);
 int check_desc(const dsq_desc *d);
-void plan_blob(const dsq_desc *d, BlobHeader *h);
+void plan_blob(const dsq_desc *d, BlobHeader *h, uint32_t flags = 0);
 int parse_blob(const void *packed, size_t bytes, BlobHeader *out);
 
 // Device view of one packed matrix (pointers into the handle's device copy
@@ -25,6 +25,8 @@ struct MatrixView {
     const uint16_t *table;   // LUT: rows x 2^bits fp16
     const int32_t *row_ptr;  // rows+1
     const uint32_t *csr;     // nnz: column | fp16 value << 16
+    const uint16_t *rscale = nullptr;  // two-axis: fp16 [rows] row scales, else null
+    const uint16_t *cscale = nullptr;  // two-axis: fp16 [cols] column scales, else null
 };
 
 // One CTA's share of the batch-1 work: rows [r0, r1), outlier pieces

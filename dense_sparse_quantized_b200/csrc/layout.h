@@ -10,6 +10,8 @@
 //   row_ptr  int32 [rows+1]
 //   csr      uint32 [nnz]   one outlier per word: column index in bits 0..15
 //                           (cols <= 65535), fp16 value in bits 16..31
+//   rscale   two-axis blobs only: fp16 [rows], the row scales r
+//   cscale   two-axis blobs only: fp16 [cols], the column scales c
 //
 // Row record.  The columns of a row are cut into S = ceil(cols/32) "slots"
 // of 32 consecutive columns; the tail slot is padded with code 0 (and, in
@@ -56,6 +58,7 @@
 namespace dsq {
 
 constexpr char kMagic[8] = {'D', 'S', 'Q', 'B', 'L', 'O', 'B', '1'};
+constexpr uint32_t kFlagTwoAxis = 1;  // header flag: the blob holds row and column scales
 constexpr uint32_t kVersion = 1;
 constexpr uint32_t kHeaderBytes = 256;
 constexpr uint64_t kSectionAlign = 256;
@@ -71,7 +74,9 @@ struct BlobHeader {
     int32_t slots;      // S
     int32_t row_words;  // u32 words per row record (multiple of 4)
     uint64_t off_dense, off_table, off_row_ptr, off_csr, reserved0, total;
-    uint8_t reserved[kHeaderBytes - 8 - 4 - 4 - 16 - 8 - 8 - 48];
+    uint64_t off_rscale, off_cscale;  // two-axis blobs; 0 otherwise
+    uint32_t flags, pad0;
+    uint8_t reserved[kHeaderBytes - 8 - 4 - 4 - 16 - 8 - 8 - 48 - 24];
 };
 static_assert(sizeof(BlobHeader) == kHeaderBytes, "header size");
 

@@ -40,7 +40,7 @@ int check_desc(const dsq_desc *d) {
     return DSQ_OK;
 }
 
-void plan_blob(const dsq_desc *d, BlobHeader *h) {
+void plan_blob(const dsq_desc *d, BlobHeader *h, uint32_t flags) {
     memset(h, 0, sizeof(*h));
     memcpy(h->magic, kMagic, sizeof(kMagic));
     h->version = kVersion;
@@ -65,6 +65,13 @@ void plan_blob(const dsq_desc *d, BlobHeader *h) {
     h->off_csr = off;
     // +16: kernels copy 16-byte-aligned spans, up to 12 bytes past the end
     off = align_up(off + (uint64_t)d->nnz * 4 + 16, kSectionAlign);
+    h->flags = flags;
+    if (flags & kFlagTwoAxis) {
+        h->off_rscale = off;
+        off = align_up(off + (uint64_t)d->rows * 2, kSectionAlign);
+        h->off_cscale = off;
+        off = align_up(off + (uint64_t)d->cols * 2 + 16, kSectionAlign);
+    }
     h->total = off;
 }
 
@@ -73,16 +80,17 @@ int parse_blob(const void *packed, size_t bytes, BlobHeader *out) {
     BlobHeader h;
     memcpy(&h, packed, sizeof(h));
     if (memcmp(h.magic, kMagic, sizeof(kMagic)) != 0 || h.version != kVersion ||
-        h.header_bytes != kHeaderBytes)
+        h.header_bytes != kHeaderBytes || (h.flags & ~kFlagTwoAxis) != 0)
         return DSQ_ERR_INVALID_ARG;
     dsq_desc d = {h.rows, h.cols, h.bits, h.mode, h.nnz};
     int rc = check_desc(&d);
     if (rc != DSQ_OK) return rc;
     BlobHeader want;
-    plan_blob(&d, &want);
+    plan_blob(&d, &want, h.flags);
     if (want.slots != h.slots || want.row_words != h.row_words || want.off_dense != h.off_dense ||
         want.off_table != h.off_table || want.off_row_ptr != h.off_row_ptr ||
-        want.off_csr != h.off_csr || h.reserved0 != 0 || want.total != h.total || h.total > bytes)
+        want.off_csr != h.off_csr || h.reserved0 != 0 || want.off_rscale != h.off_rscale ||
+        want.off_cscale != h.off_cscale || want.total != h.total || h.total > bytes)
         return DSQ_ERR_INVALID_ARG;
     *out = h;
     return DSQ_OK;
@@ -122,9 +130,10 @@ int check_blob_contents(const void *packed, const BlobHeader &h) {
 
 using namespace dsq;
 
-extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t *table,
-                        const uint16_t *zeros, const int32_t *row_ptr, const int32_t *col_idx,
-                        const uint16_t *values, void *out, size_t *out_bytes) {
+static int pack_impl(const dsq_desc *d, const uint8_t *codes, const uint16_t *table, const uint16_t *zeros,
+                     const int32_t *row_ptr, const int32_t *col_idx, const uint16_t *values,
+                     const uint16_t *rscale, const uint16_t *cscale, uint32_t flags, void *out,
+                     size_t *out_bytes) {
     if (!out_bytes) return DSQ_ERR_INVALID_ARG;
     int rc = check_desc(d);
     if (rc != DSQ_OK) return rc;
@@ -187,9 +196,16 @@ extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t 
     }
     for (int64_t k = 0; k < nnz; k++)
         if (!isfinite(half_bits_to_double(values[k]))) return DSQ_ERR_INVALID_ARG;
+    if (flags & kFlagTwoAxis) {
+        if ((M > 0 && !rscale) || (N > 0 && !cscale)) return DSQ_ERR_INVALID_ARG;
+        for (int64_t i = 0; i < M; i++)
+            if (!isfinite(half_bits_to_double(rscale[i]))) return DSQ_ERR_INVALID_ARG;
+        for (int64_t j = 0; j < N; j++)
+            if (!isfinite(half_bits_to_double(cscale[j]))) return DSQ_ERR_INVALID_ARG;
+    }
 
     BlobHeader h;
-    plan_blob(d, &h);
+    plan_blob(d, &h, flags);
     if (!out || *out_bytes < h.total) {
         *out_bytes = h.total;
         return DSQ_ERR_BUFFER_TOO_SMALL;
@@ -235,7 +251,25 @@ extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t 
     else memset(blob + h.off_row_ptr, 0, 4);
     uint32_t *csr = (uint32_t *)(blob + h.off_csr);
     for (int64_t k = 0; k < nnz; k++) csr[k] = (uint32_t)(uint16_t)col_idx[k] | ((uint32_t)values[k] << 16);
+    if (flags & kFlagTwoAxis) {
+        if (M > 0) memcpy(blob + h.off_rscale, rscale, (size_t)M * 2);
+        if (N > 0) memcpy(blob + h.off_cscale, cscale, (size_t)N * 2);
+    }
     return DSQ_OK;
+}
+
+extern "C" int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t *table,
+                        const uint16_t *zeros, const int32_t *row_ptr, const int32_t *col_idx,
+                        const uint16_t *values, void *out, size_t *out_bytes) {
+    return pack_impl(d, codes, table, zeros, row_ptr, col_idx, values, nullptr, nullptr, 0, out, out_bytes);
+}
+
+extern "C" int dsq_pack_two_axis(const dsq_desc *d, const uint8_t *codes, const uint16_t *table,
+                                 const uint16_t *zeros, const int32_t *row_ptr, const int32_t *col_idx,
+                                 const uint16_t *values, const uint16_t *row_scale, const uint16_t *col_scale,
+                                 void *out, size_t *out_bytes) {
+    return pack_impl(d, codes, table, zeros, row_ptr, col_idx, values, row_scale, col_scale, kFlagTwoAxis, out,
+                     out_bytes);
 }
 
 extern "C" int dsq_blob_desc(const void *packed, size_t bytes, dsq_desc *out) {

@@ -737,7 +737,9 @@ int run_tc(const MatrixView &m, const Split &sp, const int32_t *split_start, int
 constexpr int kTcMinBatch = 3, kTcMinBatchHeavy = 16, kHeavyRowNnz = 256;
 
 bool tc_covers(const dsq_handle_s *h, int batch) {
-    return h->tc.ready && batch >= h->tc.min_batch && tc_shape_ok(h->view);
+    // two-axis matrices need x times the column scales exactly (fp32), which
+    // an fp16 B operand cannot hold
+    return h->tc.ready && batch >= h->tc.min_batch && tc_shape_ok(h->view) && !h->view.cscale;
 }
 
 int tc_launch_count(const dsq_handle_s *h, int batch) { return tc_covers(h, batch) ? (batch + 63) / 64 : -1; }

@@ -116,6 +116,30 @@ DSQ_API int dsq_pack(const dsq_desc *d, const uint8_t *codes, const uint16_t *ta
              size_t *out_bytes);
 
 /*
+ * dsq_pack_two_axis -- dsq_pack for a matrix with two-axis scales (SINQ
+ * page, "Mise a l'echelle sur deux axes"): a scale per output row and a
+ * scale per input column around the quantized dense part,
+ *
+ *     What[i][j] = r[i] * c[j] * W_dense[i][j] + W_sparse[i][j],
+ *
+ * the product evaluated exactly (not rounded to fp16) and the outliers
+ * unscaled.  Arguments as for dsq_pack, plus
+ *   row_scale  host fp16 [rows], finite (may be NULL when rows == 0);
+ *   col_scale  host fp16 [cols], finite (may be NULL when cols == 0).
+ * The blob records the scales; dsq_create, dsq_gemv and dsq_decode take it
+ * like any other (dsq_decode still writes W_dense, unscaled).  Every mode
+ * is accepted; at batch 1 table and bit-plane matrices run the tuned table
+ * kernel (x times c formed exactly in fp32 as it is loaded, r applied to
+ * each row's dense sum before the outliers are added), other shapes and
+ * batches the one-warp-per-row kernel.  Returns as dsq_pack, and
+ * DSQ_ERR_INVALID_ARG for a non-finite or missing scale.
+ */
+DSQ_API int dsq_pack_two_axis(const dsq_desc *d, const uint8_t *codes, const uint16_t *table,
+                              const uint16_t *zeros, const int32_t *row_ptr, const int32_t *col_idx,
+                              const uint16_t *values, const uint16_t *row_scale,
+                              const uint16_t *col_scale, void *out, size_t *out_bytes);
+
+/*
  * dsq_blob_desc -- read the shape of a packed blob (host).  Returns
  * DSQ_ERR_INVALID_ARG when the blob is not one dsq_pack wrote.
  */

@@ -68,6 +68,7 @@ class Problem:
     col_idx int32  [nnz]                 CSR column indices, increasing per row
     values  uint16 [nnz]                 CSR fp16 outlier values
     x       uint16 [batch, cols]         fp16 activations
+    row_scale, col_scale  uint16 [rows] / [cols] fp16 two-axis scales, or None
     """
     name: str
     rows: int
@@ -81,6 +82,8 @@ class Problem:
     col_idx: np.ndarray
     values: np.ndarray
     x: np.ndarray
+    row_scale: Optional[np.ndarray] = None
+    col_scale: Optional[np.ndarray] = None
 
     @property
     def nnz(self) -> int:
@@ -106,6 +109,8 @@ class Problem:
         else:
             meta = self.rows * (self.cols // GROUP) * 4
         csr = self.nnz * 6 + (self.rows + 1) * 4
+        if self.row_scale is not None:
+            meta += (self.rows + self.cols) * 2
         return codes + meta + csr + b * self.cols * 2 + b * self.rows * 2
 
 
@@ -261,16 +266,43 @@ def _quantize_bitplane(Wd: np.ndarray, hole: np.ndarray, bits: int):
 
 # ---------------------------------------------------------------- assembly
 
+def _two_axis_scales(Wd: np.ndarray, hole: np.ndarray, iters: int = 8):
+    """Row and column scales that even out the spread of the dense weights
+    (SINQ page, "Sinkhorn-Knopp": alternate normalisations of the rows' and
+    the columns' standard deviations).  Returns the fp16 scales and the
+    matrix divided by them."""
+    keep = ~hole
+    n_r = np.maximum(keep.sum(axis=1), 1)
+    n_c = np.maximum(keep.sum(axis=0), 1)
+    r = np.ones(Wd.shape[0])
+    c = np.ones(Wd.shape[1])
+    for _ in range(iters):
+        A = np.where(keep, Wd / np.outer(r, c), 0.0)
+        sr = np.sqrt((A * A).sum(axis=1) / n_r)
+        r *= np.where(sr > 0, sr, 1.0)
+        A = np.where(keep, Wd / np.outer(r, c), 0.0)
+        sc = np.sqrt((A * A).sum(axis=0) / n_c)
+        c *= np.where(sc > 0, sc, 1.0)
+    r16, c16 = f16_bits(r), f16_bits(c)
+    rv = r16.view(np.float16).astype(np.float64)
+    cv = c16.view(np.float16).astype(np.float64)
+    return r16, c16, np.where(hole, 0.0, Wd / np.outer(rv, cv))
+
+
 def make_problem(rows: int, cols: int, bits: int, mode: str, density: float,
                  outliers: str = "uniform", seed: int = 0, batch: int = 1,
-                 name: str = "") -> Problem:
+                 name: str = "", two_axis: bool = False) -> Problem:
     """Build one layer: outlier kind is 'topk', 'uniform', 'structured',
-    'zipf' or 'none'."""
+    'zipf' or 'none'.  two_axis: the weights carry log-normal row and column
+    gains, and the dense part is quantized after dividing out two-axis
+    scales, which the problem then holds."""
     if cols % GROUP:
         raise ValueError("cols must be a multiple of 16")
     M, N = rows, cols
     rng = np.random.default_rng(seed)
     W = rng.normal(0.0, 0.02, size=(M, N))
+    if two_axis:
+        W *= np.outer(np.exp(rng.normal(0.0, 0.5, M)), np.exp(rng.normal(0.0, 0.5, N)))
     nnz = round_half_up(density * M * N) if outliers != "none" else 0
     Wf = W.reshape(-1)
     if nnz == 0:
@@ -301,6 +333,9 @@ def make_problem(rows: int, cols: int, bits: int, mode: str, density: float,
     hole.reshape(-1)[pos] = True
     Wd = np.where(hole, 0.0, W)
     del W, Wf
+    row_scale = col_scale = None
+    if two_axis:
+        row_scale, col_scale, Wd = _two_axis_scales(Wd, hole)
     if mode == LUT:
         codes, table = _quantize_lut(Wd, hole, bits)
         zeros = None
@@ -316,7 +351,7 @@ def make_problem(rows: int, cols: int, bits: int, mode: str, density: float,
     x = f16_bits(rng.normal(0.0, 1.0, size=(batch, N)))
     return Problem(name=name, rows=M, cols=N, bits=bits, mode=mode, codes=codes,
                    table=table, zeros=zeros, row_ptr=row_ptr, col_idx=col_idx,
-                   values=values, x=x)
+                   values=values, x=x, row_scale=row_scale, col_scale=col_scale)
 
 
 # ---------------------------------------------------------------- the five workloads
@@ -345,6 +380,10 @@ CONFIGS: Dict[str, dict] = {
     "bp3": dict(rows=11008, cols=4096, bits=3, mode=BITPLANE, density=0.01,
                 outliers="uniform", seed=53, batches=(1, 2, 4),
                 about="11008x4096 3-bit-plane BPDQ (groups of 256, 4 fp16 coefficients), 1% uniform outliers"),
+    # SINQ two-axis scales around a non-uniform 3-bit table, same shape
+    "sq3": dict(rows=11008, cols=4096, bits=3, mode=LUT, density=0.01,
+                outliers="uniform", seed=60, batches=(1, 2), two_axis=True,
+                about="11008x4096 3-bit row-LUT with SINQ two-axis fp16 scales, 1% uniform outliers"),
 }
 
 
@@ -367,7 +406,7 @@ def make_config(name: str, batch: Optional[int] = None) -> Problem:
     c = CONFIGS[name]
     b = max(c["batches"]) if batch is None else batch
     return make_problem(c["rows"], c["cols"], c["bits"], c["mode"], c["density"],
-                        c["outliers"], c["seed"], b, name)
+                        c["outliers"], c["seed"], b, name, c.get("two_axis", False))
 
 
 def describe(name: str) -> str:

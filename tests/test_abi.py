@@ -295,6 +295,38 @@ def test_bitplane_pack_rejects():
     assert pack_status(pb, table=big) == dsq.DSQ_ERR_INVALID_ARG
 
 
+def test_two_axis_blob_sections_and_checks():
+    """Two-axis blobs carry the row and column scales in their own sections,
+    flagged in the header; bad scales are refused; a plain blob reader of
+    the same shape (the no-allocation entry point) refuses the larger blob
+    before touching a device."""
+    p = synth.make_problem(9, 256, 3, "lut", 0.03, "uniform", 4, 1, two_axis=True)
+    blob = dsq.pack_problem(p)
+    plain = dsq.pack(p.rows, p.cols, p.bits, p.mode, p.codes, p.table, p.zeros, p.row_ptr, p.col_idx, p.values)
+    assert len(blob) > len(plain)
+    off_rs, off_cs = (int(v) for v in np.frombuffer(blob[96:112], np.uint64))
+    flags = int(np.frombuffer(blob[112:116], np.uint32)[0])
+    assert flags == 1 and int(np.frombuffer(plain[112:116], np.uint32)[0]) == 0
+    assert np.array_equal(np.frombuffer(blob[off_rs:off_rs + 2 * p.rows], np.uint16), p.row_scale)
+    assert np.array_equal(np.frombuffer(blob[off_cs:off_cs + 2 * p.cols], np.uint16), p.col_scale)
+    codes, table, _, rp, ci, va = unpack_blob(blob)
+    assert np.array_equal(codes, p.codes) and np.array_equal(table, p.table)
+    d = dsq.blob_desc(blob)
+    assert (d.rows, d.cols, d.bits, d.mode) == (9, 256, 3, 0)
+    bad = bytearray(blob)
+    bad[112:116] = np.array([2], np.uint32).tobytes()     # an unknown flag
+    with pytest.raises(dsq.DSQError):
+        dsq.blob_desc(bytes(bad))
+    for rs, cs in ((np.full(9, 0x7E00, np.uint16), p.col_scale), (p.row_scale, np.full(256, 0x7C00, np.uint16))):
+        with pytest.raises(dsq.DSQError) as e:
+            dsq.pack(p.rows, p.cols, p.bits, p.mode, p.codes, p.table, p.zeros, p.row_ptr, p.col_idx,
+                     p.values, rs, cs)
+        assert e.value.status == dsq.DSQ_ERR_INVALID_ARG
+    lib = dsq.library()
+    desc = dsq.Desc(p.rows, p.cols, p.bits, dsq.MODE_LUT_ROW, p.nnz)
+    assert lib.dsq_gemv_noalloc(ctypes.byref(desc), 256, len(blob), 16, 16, 16, None) == dsq.DSQ_ERR_INVALID_ARG
+
+
 def test_three_bit_fields():
     """3-bit placement: columns 2j and 2j+1 of a word's ten sit 16 bits apart
     (one mask puts both into the two 16-bit halves); every pair lies in bits

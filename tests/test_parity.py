@@ -139,6 +139,36 @@ def test_bitplane_small_shapes(orc, bits, rows, cols):
             check_y(y, y_ref, bound, f"{rows}x{cols} bitplane k={bits} B={batch}")
 
 
+@pytest.mark.parametrize("batch", [1, 2])
+def test_gemv_two_axis_every_row(orc, batch):
+    """SINQ two-axis scales around a 3-bit table matrix (11008 x 4096): the
+    batch-1 table kernel with x times c formed in fp32 and r applied per
+    row; every row against the oracle; the decode is the unscaled W_dense."""
+    p, h = config("sq3")
+    if batch == 1:
+        assert np.array_equal(to_bits(h.decode()), orc.decode(p))
+    xb = synth.f16_bits(np.random.default_rng(70 + batch).standard_normal((batch, p.cols)))
+    y = gemv(h, xb, batch)
+    y_ref, bound = oracle_all_rows(orc, p, xb)
+    check_y(y, y_ref, bound, f"sq3 B={batch}")
+
+
+@pytest.mark.parametrize("bits,mode,cols", [(3, "lut", 1024), (4, "lut", 512), (3, "affine", 1024),
+                                            (4, "affine", 512), (2, "bitplane", 512), (3, "bitplane", 1024),
+                                            (3, "lut", 25600)])
+def test_two_axis_all_modes(orc, bits, mode, cols):
+    """Two-axis scales on every mode and through every path that serves them
+    (batch-1 table kernel, the generic kernel for affine matrices, past 24
+    column warps and for more rows), batches 1-3 and 9."""
+    p = synth.make_problem(37, cols, bits, mode, 0.02, "uniform", bits + cols, 9, two_axis=True)
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        assert np.array_equal(to_bits(h.decode()), orc.decode(p))
+        for batch in (1, 2, 3, 9):
+            y = gemv(h, p.x, batch)
+            y_ref, bound = orc.gemv(p, x=p.x[:batch])
+            check_y(y, y_ref, bound, f"two-axis {bits} {mode} {cols} B={batch}")
+
+
 @pytest.mark.parametrize("name", C4)
 @pytest.mark.parametrize("batch", [1, 16])
 def test_gemv_c4_every_row(orc, name, batch):
