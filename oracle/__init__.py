@@ -54,6 +54,8 @@ class Oracle:
         lib.oracle_gemv_rows.restype = _I
         lib.oracle_gemv_rows.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I,
                                          _P, _P, _I, _P, _P]
+        lib.oracle_decompose.restype = _I
+        lib.oracle_decompose.argtypes = [_I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, _P]
         lib.oracle_materialize_two_axis.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                                                     _P, _P, _P]
         lib.oracle_gemv_rows_two_axis.restype = _I
@@ -131,6 +133,30 @@ class Oracle:
         if rc != 0:
             raise MemoryError("oracle_gemv_rows failed")
         return y, bound
+
+
+    # -- the decomposition before the product -------------------------
+    def decompose(self, w: np.ndarray, bits: int, mode: str, nnz: int):
+        """Outliers (the nnz largest |w|) and the quantized dense part of fp32
+        weights w [rows, cols]: (codes, table, zeros, row_ptr, col_idx,
+        values) as dsq_pack takes them."""
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        rows, cols = w.shape
+        m = {"lut": 0, "affine": 1}[mode]
+        codes = np.empty((rows, cols), np.uint8)
+        if m == 0:
+            table, zeros = np.empty((rows, 1 << bits), np.uint16), None
+        else:
+            table, zeros = np.empty((rows, cols // 16), np.uint16), np.empty((rows, cols // 16), np.uint16)
+        rp = np.empty(rows + 1, np.int32)
+        ci = np.empty(max(nnz, 1), np.int32)
+        va = np.empty(max(nnz, 1), np.uint16)
+        rc = self.lib.oracle_decompose(rows, cols, bits, m, nnz, w.ctypes.data, codes.ctypes.data,
+                                       table.ctypes.data, None if zeros is None else zeros.ctypes.data,
+                                       rp.ctypes.data, ci.ctypes.data, va.ctypes.data)
+        if rc != 0:
+            raise MemoryError("oracle_decompose failed")
+        return codes, table, zeros, rp, ci[:nnz], va[:nnz]
 
 
 _default: Optional[Oracle] = None

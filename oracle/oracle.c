@@ -284,3 +284,150 @@ int oracle_gemv(int rows, int cols, int bits, int mode, const uint8_t *codes,
                             row_ptr, col_idx, values, batch, x, NULL, rows,
                             y_ref, bound);
 }
+
+/* ------------------------------------------------------------------------
+ * The decomposition before the product (SqueezeLLM page, "Dense-and-Sparse
+ * decomposition"; SpQR page, "Diagramme de la matrice sparse vs dense" and
+ * "Quantification d'un modele"): from the weights w (fp32, rows x cols) the
+ * nnz largest |w| of the whole matrix become fp16 outliers in CSR (equal |w|:
+ * the lower row-major index first); the other weights form the dense part,
+ * the outlier positions being holes that count as 0, quantized
+ *  - AFFINE: per group of 16 inputs, over the range [min, max] of its dense
+ *    weights widened to contain 0: scale = fp16((max - min) / (2^b - 1));
+ *    when that scale is not a positive finite number the group gets scale 1
+ *    and zero 0; zero = rint(-min / scale), clipped to [0, 2^b - 1];
+ *    q = rint(w / scale) + zero, clipped the same way (rint: nearest, ties to
+ *    even; the arithmetic in fp64 on the fp16 scale);
+ *  - LUT: per row, the centroids are the fp16 roundings of the odd quantiles
+ *    (2k+1)/2^(b+1) of the row's dense (non-hole) weights, a quantile being
+ *    the linear interpolation x[lo] + t (x[lo+1] - x[lo]) at position
+ *    (n-1) p of the sorted values (0 when the row has none); each weight, a
+ *    hole counting as 0, takes the nearest centroid, the lower index on a tie.
+ * ---------------------------------------------------------------------- */
+
+struct oracle_item {
+    float a;
+    int64_t i;
+};
+
+static int oracle_cmp_outlier(const void *pa, const void *pb)
+{
+    const struct oracle_item *a = (const struct oracle_item *)pa;
+    const struct oracle_item *b = (const struct oracle_item *)pb;
+    if (a->a != b->a)
+        return a->a > b->a ? -1 : 1;
+    return a->i < b->i ? -1 : (a->i > b->i ? 1 : 0);
+}
+
+static int oracle_cmp_double(const void *pa, const void *pb)
+{
+    double a = *(const double *)pa, b = *(const double *)pb;
+    return a < b ? -1 : (a > b ? 1 : 0);
+}
+
+int oracle_decompose(int rows, int cols, int bits, int mode, int64_t nnz,
+                     const float *w, uint8_t *codes, uint16_t *table,
+                     uint16_t *zeros, int32_t *row_ptr, int32_t *col_idx,
+                     uint16_t *values)
+{
+    int64_t n = (int64_t)rows * cols, k = 0;
+    int K = 1 << bits, qmax = K - 1;
+    struct oracle_item *it = (struct oracle_item *)malloc(sizeof(*it) * (n > 0 ? n : 1));
+    uint8_t *hole = (uint8_t *)calloc(n > 0 ? n : 1, 1);
+    double *sorted = (double *)malloc(sizeof(double) * (cols > 0 ? cols : 1));
+    if (!it || !hole || !sorted || nnz < 0 || nnz > n) {
+        free(it);
+        free(hole);
+        free(sorted);
+        return -1;
+    }
+    /* outliers: the nnz largest |w| */
+    for (int64_t t = 0; t < n; t++) {
+        it[t].a = fabsf(w[t]);
+        it[t].i = t;
+    }
+    qsort(it, (size_t)n, sizeof(*it), oracle_cmp_outlier);
+    for (int64_t t = 0; t < nnz; t++)
+        hole[it[t].i] = 1;
+    /* CSR, row by row, columns ascending */
+    row_ptr[0] = 0;
+    for (int64_t i = 0; i < rows; i++) {
+        for (int64_t j = 0; j < cols; j++)
+            if (hole[i * cols + j]) {
+                col_idx[k] = (int32_t)j;
+                values[k] = oracle_double_to_half((double)w[i * cols + j]);
+                k++;
+            }
+        row_ptr[i + 1] = (int32_t)k;
+    }
+    /* dense part */
+    if (mode == ORACLE_AFFINE) {
+        int64_t G = cols / ORACLE_GROUP;
+        for (int64_t i = 0; i < rows; i++)
+            for (int64_t g = 0; g < G; g++) {
+                double mn = 0.0, mx = 0.0, sv, z;
+                uint16_t s16;
+                for (int c = 0; c < ORACLE_GROUP; c++) {
+                    int64_t t = i * cols + g * ORACLE_GROUP + c;
+                    double v = hole[t] ? 0.0 : (double)w[t];
+                    if (v < mn) mn = v;
+                    if (v > mx) mx = v;
+                }
+                s16 = oracle_double_to_half((mx - mn) / qmax);
+                sv = oracle_half_to_double(s16);
+                if (isfinite(sv) && sv > 0.0) {
+                    z = rint(-mn / sv);
+                    z = z < 0.0 ? 0.0 : (z > qmax ? qmax : z);
+                } else {
+                    s16 = 0x3C00;
+                    sv = 1.0;
+                    z = 0.0;
+                }
+                table[i * G + g] = s16;
+                zeros[i * G + g] = oracle_double_to_half(z);
+                for (int c = 0; c < ORACLE_GROUP; c++) {
+                    int64_t t = i * cols + g * ORACLE_GROUP + c;
+                    double v = hole[t] ? 0.0 : (double)w[t];
+                    double q = rint(v / sv) + z;
+                    codes[t] = (uint8_t)(q < 0.0 ? 0 : (q > qmax ? qmax : q));
+                }
+            }
+    } else {
+        for (int64_t i = 0; i < rows; i++) {
+            int64_t m = 0;
+            double cent[16];
+            for (int64_t j = 0; j < cols; j++)
+                if (!hole[i * cols + j])
+                    sorted[m++] = (double)w[i * cols + j];
+            qsort(sorted, (size_t)m, sizeof(double), oracle_cmp_double);
+            for (int q = 0; q < K; q++) {
+                double c = 0.0;
+                if (m > 0) {
+                    double p = (2.0 * q + 1.0) / (2.0 * K);
+                    double h = (double)(m - 1) * p;
+                    int64_t lo = (int64_t)floor(h);
+                    int64_t hi = lo + 1 < m ? lo + 1 : m - 1;
+                    c = sorted[lo] + (h - (double)lo) * (sorted[hi] - sorted[lo]);
+                }
+                table[i * K + q] = oracle_double_to_half(c);
+                cent[q] = oracle_half_to_double(table[i * K + q]);
+            }
+            for (int64_t j = 0; j < cols; j++) {
+                int64_t t = i * cols + j;
+                double v = hole[t] ? 0.0 : (double)w[t];
+                int best = 0;
+                double bd = fabs(v - cent[0]);
+                for (int q = 1; q < K; q++)
+                    if (fabs(v - cent[q]) < bd) {
+                        bd = fabs(v - cent[q]);
+                        best = q;
+                    }
+                codes[t] = (uint8_t)best;
+            }
+        }
+    }
+    free(it);
+    free(hole);
+    free(sorted);
+    return 0;
+}
