@@ -49,6 +49,8 @@ def parse_args(argv=None):
     ap.add_argument("--config", default="c2")
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", default="dsq", choices=["dsq", "reference"])
+    ap.add_argument("--op", default="gemv", choices=["gemv", "decompose"],
+                    help="decompose: time the on-device decomposition of the config's weights instead")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     return ap.parse_args(argv)
@@ -510,10 +512,74 @@ def run_dsq(args):
     return 0
 
 
+def run_decompose(args):
+    """The step before the product on one GPU: dsq_decompose of the config's
+    shape from fp32 weights (N(0, 0.02^2) plus Laplace spikes) resident in
+    HBM, the outlier count of the config, K timed calls between CUDA events."""
+    import torch
+    import dense_sparse_quantized_b200 as dsq
+    import synth
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    c = synth.CONFIGS[args.config]
+    if c["mode"] not in ("lut", "affine"):
+        raise SystemExit("decompose covers table and affine configs")
+    M, N, bits, mode = c["rows"], c["cols"], c["bits"], c["mode"]
+    nnz = synth.round_half_up(c["density"] * M * N)
+    w = torch.from_numpy(synth.spiky_weights(M, N, c["density"], c["seed"])).cuda()
+    out = dsq.decompose(w, bits, mode, nnz)          # allocates outputs and workspace once
+    ws_bytes = ctypes_workspace_bytes(dsq, M, N, bits, mode, nnz)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=w.device)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            dsq.decompose(w, bits, mode, nnz, stream=stream, workspace=ws)
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks, torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            dsq.decompose(w, bits, mode, nnz, stream=stream, workspace=ws)
+        e1.record(stream)
+        e1.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    table_b = M * (1 << bits) * 2 if mode == "lut" else M * (N // 16) * 4
+    alg = 4 * M * N + M * N + table_b + 6 * nnz + 4 * (M + 1)
+    peak, peak_src = measured_peaks()
+    line = {"metric": "on-device dense-and-sparse decomposition: us per matrix, GB/s on W read once + arrays written",
+            "value": alg / (us * 1e-6) / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": us / 1e3, "us_per_call": us, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 in / f64 quantizer arithmetic",
+            "data": "synthetic",
+            "config": {"workload": f"{args.config} shape: {M}x{N} {mode} {bits}-bit, {nnz} outliers "
+                                   "(top |w|) from N(0,0.02^2) + Laplace(0,0.2) spikes",
+                       "rows": M, "cols": N, "bits": bits, "mode": mode, "nnz": nnz,
+                       "algorithmic_bytes": alg, "launches_per_call": 9 if nnz else 3,
+                       "l2": "W (fp32) is %d MB; it is read by several passes per call" % (4 * M * N // 10**6)},
+            "roofline": {"bound": "hbm", "achieved": alg / (us * 1e-6) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": alg / (us * 1e-6) / 1e9 / peak, "traffic": None,
+                         "peak_source": peak_src},
+            "clocks": clocks.summary()}
+    del out
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def ctypes_workspace_bytes(dsq, M, N, bits, mode, nnz):
+    import ctypes
+    d = dsq.Desc(M, N, bits, dsq.MODE_LUT_ROW if mode == "lut" else dsq.MODE_AFFINE_G16, nnz)
+    size = ctypes.c_size_t(0)
+    dsq.library().dsq_decompose(ctypes.byref(d), None, None, None, None, None, None, None, None,
+                                ctypes.byref(size), None)
+    return size.value
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "decompose":
+        return run_decompose(args)
     return run_dsq(args)
 
 

@@ -34,7 +34,7 @@ MODE_BITPLANE = 2
 
 EXPORTS = ("dsq_pack", "dsq_pack_two_axis", "dsq_blob_desc", "dsq_create", "dsq_gemv", "dsq_gemv_launches", "dsq_decode",
            "dsq_handle_desc", "dsq_device_bytes", "dsq_check", "dsq_destroy", "dsq_status_string",
-           "dsq_gemv_noalloc", "dsq_selftest_wait_timeout")
+           "dsq_gemv_noalloc", "dsq_selftest_wait_timeout", "dsq_decompose")
 
 
 class DSQError(RuntimeError):
@@ -75,6 +75,7 @@ def library() -> ctypes.CDLL:
         lib.dsq_destroy.argtypes = [P]
         lib.dsq_gemv_noalloc.argtypes = [ctypes.POINTER(Desc), P, SZ, P, P, I, P]
         lib.dsq_selftest_wait_timeout.argtypes = [P, P]
+        lib.dsq_decompose.argtypes = [ctypes.POINTER(Desc), P, P, P, P, P, P, P, P, ctypes.POINTER(SZ), P]
         lib.dsq_status_string.argtypes = [I]
         lib.dsq_status_string.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -273,3 +274,40 @@ def gemv_noalloc(desc: Desc, packed_device, x, y, stream=None):
                                       x.data_ptr(), y.data_ptr(), batch, _stream_ptr(stream)),
            "dsq_gemv_noalloc")
     return y
+
+
+def decompose(w, bits: int, mode: str, nnz: int, stream=None, workspace=None):
+    """Outliers and quantized dense part of device fp32 weights w [rows, cols]
+    (dsq_decompose): returns cuda tensors (codes, table, zeros or None,
+    row_ptr, col_idx, values) -- the arrays pack() takes.  ``workspace``:
+    an optional cuda uint8 tensor to reuse; one is allocated otherwise."""
+    import torch
+    if w.dtype != torch.float32 or not w.is_cuda or not w.is_contiguous() or w.dim() != 2:
+        raise ValueError("w must be a contiguous 2-D cuda float32 tensor")
+    rows, cols = w.shape
+    m = {"lut": MODE_LUT_ROW, "affine": MODE_AFFINE_G16}[mode]
+    d = Desc(rows, cols, int(bits), m, int(nnz))
+    dev = w.device
+    size = ctypes.c_size_t(0)
+    rc = library().dsq_decompose(ctypes.byref(d), None, None, None, None, None, None, None, None,
+                                 ctypes.byref(size), None)
+    if rc != DSQ_ERR_BUFFER_TOO_SMALL:
+        _check(rc, "dsq_decompose")
+    if workspace is None or workspace.numel() < size.value:
+        workspace = torch.empty(max(size.value, 1), dtype=torch.uint8, device=dev)
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+    if m == MODE_LUT_ROW:
+        table = torch.empty((rows, 1 << bits), dtype=torch.float16, device=dev)
+        zeros = None
+    else:
+        table = torch.empty((rows, cols // 16), dtype=torch.float16, device=dev)
+        zeros = torch.empty((rows, cols // 16), dtype=torch.float16, device=dev)
+    row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(nnz, 1), dtype=torch.int32, device=dev)
+    values = torch.empty(max(nnz, 1), dtype=torch.float16, device=dev)
+    size = ctypes.c_size_t(workspace.numel())
+    _check(library().dsq_decompose(ctypes.byref(d), w.data_ptr(), codes.data_ptr(), table.data_ptr(),
+                                   None if zeros is None else zeros.data_ptr(), row_ptr.data_ptr(),
+                                   col_idx.data_ptr(), values.data_ptr(), workspace.data_ptr(),
+                                   ctypes.byref(size), _stream_ptr(stream)), "dsq_decompose")
+    return codes, table, zeros, row_ptr, col_idx[:nnz], values[:nnz]

@@ -290,6 +290,47 @@ DSQ_API int dsq_destroy(dsq_handle_t h);
 DSQ_API int dsq_gemv_noalloc(const dsq_desc *d, const void *packed_device, size_t bytes, const void *x, void *y,
                              int batch, void *stream);
 
+/*
+ * dsq_decompose -- the step before dsq_pack, on the device: split dense fp32
+ * weights into outliers and a quantized dense part (SqueezeLLM page,
+ * "Dense-and-Sparse decomposition"; SpQR page, "Diagramme de la matrice
+ * sparse vs dense" and "Quantification d'un modele").
+ *   - outliers: the d->nnz largest |w| of the whole matrix (equal |w| taken
+ *     in row-major order), as CSR with fp16 values (rounded to nearest);
+ *   - dense part, outlier positions counting as 0:
+ *     AFFINE_G16: per group of 16 inputs, the range [min, max] widened to
+ *       contain 0; scale = fp16((max - min) / (2^bits - 1)) -- scale 1 and
+ *       zero 0 when that is not a positive finite number --, zero =
+ *       rint(-min / scale) and q = rint(w / scale) + zero, both clipped to
+ *       [0, 2^bits - 1] (rint: nearest, ties to even; fp64 arithmetic);
+ *     LUT_ROW: per row, the centroids are the fp16 roundings of the linear
+ *       quantiles (2k+1)/2^(bits+1) of the row's dense weights (0 for a row
+ *       of outliers only); every weight takes the nearest centroid, the
+ *       lower index on a tie.
+ * The outputs are exactly the logical arrays dsq_pack takes.
+ *   d          host; rows, cols, bits, mode (LUT_ROW or AFFINE_G16, bits 3
+ *              or 4), nnz = the number of outliers to keep.
+ *   w          device fp32 [rows][cols], finite, 16-byte aligned; read only.
+ *   codes      device uint8 [rows][cols], 16-byte aligned.
+ *   table      device fp16: LUT_ROW [rows][2^bits] centroids, AFFINE_G16
+ *              [rows][cols/16] scales.
+ *   zeros      device fp16 [rows][cols/16] (AFFINE_G16); NULL for LUT_ROW.
+ *   row_ptr    device int32 [rows+1]; col_idx device int32 [nnz]; values
+ *              device fp16 [nnz].
+ *   workspace  device scratch, 256-byte aligned, *workspace_bytes long, the
+ *              caller's; with workspace NULL (or too small) the call only
+ *              writes the size it needs to *workspace_bytes and returns
+ *              DSQ_ERR_BUFFER_TOO_SMALL.  About rows*cols/8 bytes.
+ *   stream     cudaStream_t as void*.  Asynchronous; nothing is allocated.
+ * Limits: rows*cols < 2^31; LUT_ROW needs cols <= 32768 (one row is sorted
+ * in shared memory).  Returns DSQ_OK, DSQ_ERR_INVALID_ARG (NULL or
+ * misaligned pointer, bad desc), DSQ_ERR_UNSUPPORTED (BITPLANE mode, sizes
+ * past the limits), DSQ_ERR_BUFFER_TOO_SMALL or DSQ_ERR_CUDA.
+ */
+DSQ_API int dsq_decompose(const dsq_desc *d, const float *w, void *codes, void *table, void *zeros,
+                          int32_t *row_ptr, int32_t *col_idx, void *values, void *workspace,
+                          size_t *workspace_bytes, void *stream);
+
 /* Static, never-NULL text for a status code. */
 DSQ_API const char *dsq_status_string(int status);
 

@@ -354,6 +354,20 @@ def make_problem(rows: int, cols: int, bits: int, mode: str, density: float,
                    values=values, x=x, row_scale=row_scale, col_scale=col_scale)
 
 
+# ---------------------------------------------------------------- raw weights
+
+def spiky_weights(rows: int, cols: int, density: float, seed: int) -> np.ndarray:
+    """Unquantized fp32 weights shaped like the workloads' (N(0, 0.02^2) plus
+    Laplace(0, 0.2) spikes at round(density * rows * cols) uniform positions),
+    the input of the on-device decomposition."""
+    rng = np.random.default_rng(seed)
+    w = rng.normal(0.0, 0.02, size=(rows, cols))
+    n = round_half_up(density * rows * cols)
+    pos = rng.choice(rows * cols, n, replace=False)
+    w.reshape(-1)[pos] += rng.laplace(0.0, 0.2, n)
+    return w.astype(np.float32)
+
+
 # ---------------------------------------------------------------- the five workloads
 
 C4_LAYERS = (("q", 6656, 6656), ("k", 6656, 6656), ("v", 6656, 6656),
