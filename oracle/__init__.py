@@ -80,8 +80,8 @@ class Oracle:
     # -- the method ----------------------------------------------------
     @staticmethod
     def _args(p):
-        mode = {"lut": 0, "affine": 1, "bitplane": 2}[p.mode]
-        codes = np.ascontiguousarray(p.codes, dtype=np.uint8)
+        mode = {"lut": 0, "affine": 1, "bitplane": 2, "intgrid": 3}[p.mode]
+        codes = np.ascontiguousarray(p.codes, dtype=np.int16 if mode == 3 else np.uint8)
         table = np.ascontiguousarray(p.table, dtype=np.uint16)
         zeros = (np.ascontiguousarray(p.zeros, dtype=np.uint16)
                  if p.zeros is not None else None)

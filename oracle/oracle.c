@@ -29,6 +29,11 @@
  *    dimension.  Read as: groups of 32 * 2^k inputs, fp16 coefficients, a
  *    weight's k plane bits held in one code q with b_i = bit (i-1) of q, and
  *    the sum C_0 + sum_i C_i b_i evaluated exactly and rounded once to fp16.
+ *  - Huffman-encoded PTQ (gist.science 2507.18553, the HPTQ bullet): inliers
+ *    and outliers on one unconstrained integer grid, the integers Huffman
+ *    coded.  Read as: an fp16 scale per group of 16 inputs and a signed
+ *    integer q per weight (|q| <= 8191), w = scale * q rounded once to fp16;
+ *    the Huffman code is storage, so the oracle reads the integers directly.
  *  - SINQ page, "Mise a l'echelle sur deux axes": a vector of scales for the
  *    rows and another for the columns around the quantized matrix.  Read as:
  *    the dense weight is r_i * c_j * Wd_ij with fp16 r and c and Wd the
@@ -56,6 +61,7 @@
 #define ORACLE_LUT 0
 #define ORACLE_AFFINE 1
 #define ORACLE_BITPLANE 2
+#define ORACLE_INTGRID 3
 #define ORACLE_GROUP 16
 
 /* IEEE 754 binary16 -> real value: sign, 5-bit biased exponent (bias 15),
@@ -124,13 +130,20 @@ void oracle_double_to_half_n(const double *v, uint16_t *out, int64_t n)
 }
 
 /* Decoded dense weight of row i, column j, as an fp16 bit pattern.
- * table: LUT mode rows x 2^bits centroids; AFFINE mode rows x cols/16 scales;
- * BITPLANE mode rows x cols/(32*2^bits) x (bits+1) coefficients C_0..C_k.
+ * codes: one uint8 code per weight; INTGRID mode: one int16 integer.
+ * table: LUT mode rows x 2^bits centroids; AFFINE and INTGRID modes rows x
+ * cols/16 scales; BITPLANE mode rows x cols/(32*2^bits) x (bits+1)
+ * coefficients C_0..C_k.
  * zeros: AFFINE mode rows x cols/16 integral zeros (unused otherwise). */
 uint16_t oracle_decode_one(int64_t i, int64_t j, int cols, int bits, int mode,
                            const uint8_t *codes, const uint16_t *table,
                            const uint16_t *zeros)
 {
+    if (mode == ORACLE_INTGRID) {
+        int qi = ((const int16_t *)codes)[i * (int64_t)cols + j];
+        double scale = oracle_half_to_double(table[i * (int64_t)(cols / ORACLE_GROUP) + j / ORACLE_GROUP]);
+        return oracle_double_to_half(scale * (double)qi);
+    }
     int q = codes[i * (int64_t)cols + j];
     if (mode == ORACLE_LUT)
         return table[i * ((int64_t)1 << bits) + q];

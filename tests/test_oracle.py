@@ -231,6 +231,31 @@ def pin_bitplane_uniform_grid_is_affine(orc):
             assert np.array_equal(orc.decode(bp), orc.decode(af)), (k, s, z)
 
 
+def pin_intgrid_decode_golden(orc):
+    """Hand-worked fp16(scale * q) on the unconstrained integer grid (the
+    Huffman-coded PTQ reading): large |q|, ties, subnormal scales."""
+    g = json.load(open(os.path.join(GOLDEN, "intgrid_decode.json")))
+    for c in g["cases"]:
+        q = np.zeros(16, np.int16)
+        q[:len(c["q"])] = c["q"]
+        p = problem(1, 16, 14, "intgrid", np.zeros(16), [[int(c["scale"], 16)]], None, [0, 0], [], [],
+                    np.zeros(16))
+        p.codes = q.reshape(1, 16)
+        got = orc.decode(p)[0, :len(c["q"])]
+        assert [hex(int(v)) for v in got] == [hex(int(v, 16)) for v in c["expect"]], c["why"]
+
+
+def pin_intgrid_group_layout(orc):
+    """Columns 16g .. 16g+15 of row r use scale [r][g]; with q in 0..7 and
+    power-of-two scales the weights are exact."""
+    q = np.tile(np.arange(48) % 8, (2, 1)).astype(np.int16)
+    scales = np_d2h([[1.0, 2.0, 0.5], [4.0, 0.25, 8.0]])
+    p = problem(2, 48, 14, "intgrid", np.zeros(96), scales, None, [0, 0, 0], [], [], np.zeros(48))
+    p.codes = q
+    want = q * np.repeat(np_h2d(scales), 16, axis=1)
+    assert np.array_equal(np_h2d(orc.decode(p)), want)
+
+
 def pin_two_axis_golden(orc):
     """The hand-worked two-axis example (SINQ page, "Mise a l'echelle sur deux
     axes"): What = r_i c_j Wd_ij plus the unscaled outliers, and its product."""
@@ -367,7 +392,7 @@ def pin_rows_subset(orc):
 PINS = [pin_half_to_double_exhaustive, pin_double_to_half, pin_csr_example,
         pin_lut_decode_identity, pin_affine_decode_golden, pin_affine_group_layout,
         pin_bitplane_decode_golden, pin_bitplane_group_layout, pin_bitplane_uniform_grid_is_affine,
-        pin_two_axis_golden, pin_two_axis_unit_scales,
+        pin_two_axis_golden, pin_two_axis_unit_scales, pin_intgrid_decode_golden, pin_intgrid_group_layout,
         pin_gemv_exact, pin_special_cases, pin_decomposition, pin_rows_subset]
 
 
@@ -413,6 +438,10 @@ MUTANTS = {
     "two_axis_col_by_row": ("double c = cscale ? oracle_half_to_double(cscale[j]) : 1.0;",
                             "double c = cscale ? oracle_half_to_double(cscale[i]) : 1.0;"),
     "two_axis_no_row_scale": ("double r = rscale ? oracle_half_to_double(rscale[i]) : 1.0;", "double r = 1.0;"),
+    "intgrid_unsigned": ("int qi = ((const int16_t *)codes)[i * (int64_t)cols + j];",
+                         "int qi = ((const uint16_t *)codes)[i * (int64_t)cols + j];"),
+    "intgrid_group_width": ("table[i * (int64_t)(cols / ORACLE_GROUP) + j / ORACLE_GROUP]);\n        return oracle_double_to_half(scale * (double)qi);",
+                            "table[i * (int64_t)(cols / ORACLE_GROUP) + j / 32]);\n        return oracle_double_to_half(scale * (double)qi);"),
     "first_column_skipped": ("for (int64_t j = 0; j < cols; j++) {\n                acc",
                              "for (int64_t j = 1; j < cols; j++) {\n                acc"),
 }
