@@ -31,8 +31,9 @@ DSQ_ERR_SCRATCH_LIMIT = -7
 MODE_LUT_ROW = 0
 MODE_AFFINE_G16 = 1
 MODE_BITPLANE = 2
+MODE_INTGRID = 3
 
-EXPORTS = ("dsq_pack", "dsq_pack_two_axis", "dsq_blob_desc", "dsq_create", "dsq_gemv", "dsq_gemv_launches", "dsq_decode",
+EXPORTS = ("dsq_pack", "dsq_pack_two_axis", "dsq_pack_intgrid", "dsq_blob_desc", "dsq_create", "dsq_gemv", "dsq_gemv_launches", "dsq_decode",
            "dsq_handle_desc", "dsq_device_bytes", "dsq_check", "dsq_destroy", "dsq_status_string",
            "dsq_gemv_noalloc", "dsq_selftest_wait_timeout", "dsq_decompose")
 
@@ -63,6 +64,7 @@ def library() -> ctypes.CDLL:
         lib.dsq_pack.argtypes = [ctypes.POINTER(Desc), P, P, P, P, P, P, P, ctypes.POINTER(SZ)]
         lib.dsq_pack_two_axis.argtypes = [ctypes.POINTER(Desc), P, P, P, P, P, P, P, P, P,
                                           ctypes.POINTER(SZ)]
+        lib.dsq_pack_intgrid.argtypes = [ctypes.POINTER(Desc), P, P, P, P, P, P, ctypes.POINTER(SZ)]
         lib.dsq_blob_desc.argtypes = [P, SZ, ctypes.POINTER(Desc)]
         lib.dsq_create.argtypes = [P, SZ, I, ctypes.POINTER(P)]
         lib.dsq_gemv.argtypes = [P, P, P, I, P]
@@ -131,9 +133,30 @@ def pack(rows: int, cols: int, bits: int, mode, codes, table, zeros, row_ptr, co
     return buf.raw[:size.value]
 
 
+def pack_intgrid(rows: int, cols: int, q, scales, row_ptr, col_idx, values) -> bytes:
+    """Huffman-code an integer-grid matrix (dsq_pack_intgrid): q int16
+    [rows, cols] (|q| <= 8191), scales fp16 bits [rows, cols/16], optional
+    outliers as CSR."""
+    lib = library()
+    nnz = int(np.asarray(row_ptr)[-1]) if row_ptr is not None and len(row_ptr) else 0
+    d = Desc(int(rows), int(cols), 14, MODE_INTGRID, nnz)
+    keep = [_arr(q, np.int16), _arr(scales, np.uint16), _arr(row_ptr, np.int32),
+            _arr(col_idx, np.int32), _arr(values, np.uint16)]
+    ptrs = [p for _, p in keep]
+    size = ctypes.c_size_t(0)
+    rc = lib.dsq_pack_intgrid(ctypes.byref(d), *ptrs, None, ctypes.byref(size))
+    if rc != DSQ_ERR_BUFFER_TOO_SMALL:
+        _check(rc, "dsq_pack_intgrid")
+    buf = ctypes.create_string_buffer(size.value)
+    _check(lib.dsq_pack_intgrid(ctypes.byref(d), *ptrs, buf, ctypes.byref(size)), "dsq_pack_intgrid")
+    return buf.raw[:size.value]
+
+
 def pack_problem(p) -> bytes:
     """pack() from an object with rows, cols, bits, mode, codes, table, zeros,
     row_ptr, col_idx, values attributes."""
+    if p.mode == "intgrid":
+        return pack_intgrid(p.rows, p.cols, p.codes, p.table, p.row_ptr, p.col_idx, p.values)
     return pack(p.rows, p.cols, p.bits, p.mode, p.codes, p.table, p.zeros, p.row_ptr,
                 p.col_idx, p.values, getattr(p, "row_scale", None), getattr(p, "col_scale", None))
 

@@ -54,6 +54,7 @@ extern "C" int dsq_create(const void *packed, size_t bytes, int device, dsq_hand
     BlobHeader hd;
     int rc = parse_blob(packed, bytes, &hd);
     if (rc == DSQ_OK) rc = check_blob_contents(packed, hd);
+    if (rc == DSQ_OK && hd.mode == DSQ_MODE_INTGRID) rc = check_intgrid_contents(packed, hd);
     if (rc != DSQ_OK) return rc;
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess) return DSQ_ERR_CUDA;
@@ -92,6 +93,10 @@ extern "C" int dsq_create(const void *packed, size_t bytes, int device, dsq_hand
     m.table = (const uint16_t *)(h->d_blob + hd.off_table);
     m.row_ptr = (const int32_t *)(h->d_blob + hd.off_row_ptr);
     m.csr = (const uint32_t *)(h->d_blob + hd.off_csr);
+    if (hd.mode == DSQ_MODE_INTGRID) {
+        m.slot_bits = (const uint32_t *)(h->d_blob + hd.off_index);
+        m.codebook = (const uint32_t *)(h->d_blob + hd.off_codebook);
+    }
     if (hd.flags & kFlagTwoAxis) {
         m.rscale = (const uint16_t *)(h->d_blob + hd.off_rscale);
         m.cscale = (const uint16_t *)(h->d_blob + hd.off_cscale);
@@ -127,6 +132,7 @@ extern "C" int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void 
     const __half *xh = (const __half *)x;
     __half *yh = (__half *)y;
     const cudaStream_t st = (cudaStream_t)stream;
+    if (h->view.mode == DSQ_MODE_INTGRID) return launch_gemv_intgrid(h, xh, yh, batch, st);
     // tensor cores where they cover the shape and batch; else the tuned
     // batch-1 kernel once per activation row; else the generic kernel
     int rc = launch_gemv_tc(h, xh, yh, batch, st);
@@ -142,6 +148,7 @@ extern "C" int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void 
 
 extern "C" int dsq_gemv_launches(dsq_handle_t h, int batch) {
     if (!h || batch < 1) return -1;
+    if (h->view.mode == DSQ_MODE_INTGRID) return gemv_launch_count(h, batch);
     int n = tc_launch_count(h, batch);
     if (n < 0 && batch > 1) n = batched_launch_count(h, batch);
     if (n < 0 && fused_launch_count(h, 1) > 0) n = batch * fused_launch_count(h, 1);
@@ -152,6 +159,7 @@ extern "C" int dsq_decode(dsq_handle_t h, void *w_dense_out, void *stream) {
     if (!h || !w_dense_out) return DSQ_ERR_INVALID_ARG;
     DeviceGuard guard(h->device);
     if (!guard.ok) return DSQ_ERR_CUDA;
+    if (h->view.mode == DSQ_MODE_INTGRID) return launch_decode_intgrid(h, (__half *)w_dense_out, (cudaStream_t)stream);
     return launch_decode(h, (__half *)w_dense_out, (cudaStream_t)stream);
 }
 

@@ -822,7 +822,7 @@ bn_lut_kernel(B1Params p, const __half *__restrict__ x, __half *__restrict__ y, 
 enum Kind { kNone = -1, kAff3 = 0, kLut3 = 3, kLut4 = 4, kBp2 = 12, kBp3 = 13 };
 
 Kind b1_kind(const MatrixView &m, int batch) {
-    if (batch != 1 || m.rows <= 0 || m.cols <= 0) return kNone;
+    if (batch != 1 || m.rows <= 0 || m.cols <= 0 || m.mode == kModeIntGrid) return kNone;
     if ((m.slots + 31) / 32 > kMaxWarps) return kNone;
     // the affine kernel multiplies fp16 x, which cannot hold c_j x_j exactly
     if (m.mode == DSQ_MODE_AFFINE_G16) return m.bits == 3 && !m.cscale ? kAff3 : kNone;
@@ -1033,7 +1033,8 @@ int batched_launch_count(const dsq_handle_s *h, int batch) {
     B1Params p;
     size_t smem;
     const MatrixView &m = h->view;
-    if (batch < 2 || m.mode == DSQ_MODE_AFFINE_G16 || m.cscale || m.rows <= 0 || m.cols <= 0 || h->sched.n_tiles == 0 ||
+    if (batch < 2 || m.mode == DSQ_MODE_AFFINE_G16 || m.mode == kModeIntGrid || m.cscale || m.rows <= 0 ||
+        m.cols <= 0 || h->sched.n_tiles == 0 ||
         !plan_bn(h, 4, &p, &smem))
         return -1;
     return (batch + 3) / 4;

@@ -13,7 +13,8 @@ namespace dsq {
 
 double half_bits_to_double(uint16_t h);
 int check_desc(const dsq_desc *d);
-void plan_blob(const dsq_desc *d, BlobHeader *h, uint32_t flags = 0);
+void plan_blob(const dsq_desc *d, BlobHeader *h, uint32_t flags = 0, uint32_t stream_words = 0,
+               uint32_t nsym = 0);
 int parse_blob(const void *packed, size_t bytes, BlobHeader *out);
 
 // Device view of one packed matrix (pointers into the handle's device copy
@@ -27,6 +28,8 @@ struct MatrixView {
     const uint32_t *csr;     // nnz: column | fp16 value << 16
     const uint16_t *rscale = nullptr;  // two-axis: fp16 [rows] row scales, else null
     const uint16_t *cscale = nullptr;  // two-axis: fp16 [cols] column scales, else null
+    const uint32_t *slot_bits = nullptr;  // INTGRID: [rows][slots] first bit of each slot
+    const uint32_t *codebook = nullptr;   // INTGRID: canonical code tables
 };
 
 // One CTA's share of the batch-1 work: rows [r0, r1), outlier pieces
@@ -86,6 +89,10 @@ int launch_decode(const dsq_handle_s *h, __half *w, cudaStream_t stream);
 int gemv_launch_count(const dsq_handle_s *h, int batch);
 int launch_zero(__half *y, int64_t n, cudaStream_t stream);
 int launch_wait_timeout(const dsq_handle_s *h, cudaStream_t stream);
+// Huffman-coded integer grids (huffman.cu).
+int launch_gemv_intgrid(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
+int launch_decode_intgrid(const dsq_handle_s *h, __half *w, cudaStream_t stream);
+int check_intgrid_contents(const void *packed, const BlobHeader &h);
 
 // Tuned batch-1 path (fused_b1.cu).  launch_gemv_fused returns
 // DSQ_ERR_UNSUPPORTED, launching nothing, for shapes it does not cover.

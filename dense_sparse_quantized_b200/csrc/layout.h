@@ -10,6 +10,11 @@
 //   row_ptr  int32 [rows+1]
 //   csr      uint32 [nnz]   one outlier per word: column index in bits 0..15
 //                           (cols <= 65535), fp16 value in bits 16..31
+//   INTGRID (Huffman-coded integers on one grid) replaces the dense and table
+//   sections: dense = the MSB-first bitstream of all rows (stream_words u32
+//   + kStreamPad words of padding), table = fp16 scales [rows][cols/16],
+//   index = u32 [rows][S] bit offset of each slot's first code, codebook =
+//   the canonical code (see huffman.cu)
 //   rscale   two-axis blobs only: fp16 [rows], the row scales r
 //   cscale   two-axis blobs only: fp16 [cols], the column scales c
 //
@@ -59,6 +64,17 @@ namespace dsq {
 
 constexpr char kMagic[8] = {'D', 'S', 'Q', 'B', 'L', 'O', 'B', '1'};
 constexpr uint32_t kFlagTwoAxis = 1;  // header flag: the blob holds row and column scales
+constexpr int kModeIntGrid = 3;        // dsq mode of Huffman-coded integer grids
+constexpr int kHuffMaxLen = 20;        // longest code
+constexpr int kHuffFastBits = 10;      // codes this short decode with one table read
+constexpr int kStreamPad = 24;         // words after the stream: a slot's 32 codes never read past it
+constexpr int kIntGridMax = 8191;      // |q| bound: scale * q is exact in fp32
+// codebook words: [0] nsym, [1] max_len, then first code, count and first
+// symbol index per length 0..kHuffMaxLen, the fast table (entry = length << 16
+// | the integer as int16, length 0 for codes longer than kHuffFastBits), the
+// symbols (int16)
+constexpr int kCbFirst = 2, kCbCount = kCbFirst + kHuffMaxLen + 1, kCbOffset = kCbCount + kHuffMaxLen + 1;
+constexpr int kCbFast = kCbOffset + kHuffMaxLen + 1, kCbSyms = kCbFast + (1 << kHuffFastBits);
 constexpr uint32_t kVersion = 1;
 constexpr uint32_t kHeaderBytes = 256;
 constexpr uint64_t kSectionAlign = 256;
@@ -76,7 +92,11 @@ struct BlobHeader {
     uint64_t off_dense, off_table, off_row_ptr, off_csr, reserved0, total;
     uint64_t off_rscale, off_cscale;  // two-axis blobs; 0 otherwise
     uint32_t flags, pad0;
-    uint8_t reserved[kHeaderBytes - 8 - 4 - 4 - 16 - 8 - 8 - 48 - 24];
+    // INTGRID blobs (Huffman-coded integers): the slot bit offsets, the
+    // codebook, the bitstream length in words and the alphabet size
+    uint64_t off_index, off_codebook;
+    uint32_t stream_words, nsym;
+    uint8_t reserved[kHeaderBytes - 8 - 4 - 4 - 16 - 8 - 8 - 48 - 24 - 24];
 };
 static_assert(sizeof(BlobHeader) == kHeaderBytes, "header size");
 
@@ -86,6 +106,7 @@ constexpr int kAff3GroupWords = 136;  // 8 words of zero bytes + 32 slot uint4
 
 __host__ __device__ inline int row_words_of(int bits, int mode, int S) {
     int w;
+    if (mode == kModeIntGrid) return 0;  // variable length: the stream has no fixed row records
     if (mode != 1)
         w = bits * S;
     else if (bits == 3)

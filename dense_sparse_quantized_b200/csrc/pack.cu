@@ -27,9 +27,12 @@ static inline uint64_t align_up(uint64_t v, uint64_t a) { return (v + a - 1) / a
 int check_desc(const dsq_desc *d) {
     if (!d) return DSQ_ERR_INVALID_ARG;
     if (d->rows < 0 || d->cols < 0 || d->cols % kGroup != 0) return DSQ_ERR_INVALID_ARG;
-    if (d->mode != DSQ_MODE_LUT_ROW && d->mode != DSQ_MODE_AFFINE_G16 && d->mode != DSQ_MODE_BITPLANE)
+    if (d->mode != DSQ_MODE_LUT_ROW && d->mode != DSQ_MODE_AFFINE_G16 && d->mode != DSQ_MODE_BITPLANE &&
+        d->mode != DSQ_MODE_INTGRID)
         return DSQ_ERR_INVALID_ARG;
-    if (d->mode == DSQ_MODE_BITPLANE) {
+    if (d->mode == DSQ_MODE_INTGRID) {
+        if (d->bits != 14) return DSQ_ERR_INVALID_ARG;
+    } else if (d->mode == DSQ_MODE_BITPLANE) {
         if (d->bits != 2 && d->bits != 3) return DSQ_ERR_INVALID_ARG;
         if (d->cols % (32 << d->bits) != 0) return DSQ_ERR_INVALID_ARG;
     } else if (d->bits != 3 && d->bits != 4) {
@@ -40,7 +43,7 @@ int check_desc(const dsq_desc *d) {
     return DSQ_OK;
 }
 
-void plan_blob(const dsq_desc *d, BlobHeader *h, uint32_t flags) {
+void plan_blob(const dsq_desc *d, BlobHeader *h, uint32_t flags, uint32_t stream_words, uint32_t nsym) {
     memset(h, 0, sizeof(*h));
     memcpy(h->magic, kMagic, sizeof(kMagic));
     h->version = kVersion;
@@ -54,6 +57,25 @@ void plan_blob(const dsq_desc *d, BlobHeader *h, uint32_t flags) {
     h->row_words = row_words_of(d->bits, d->mode, h->slots);
     uint64_t off = kHeaderBytes;
     h->off_dense = off;
+    if (d->mode == DSQ_MODE_INTGRID) {
+        // bitstream, scales, slot offsets, codebook
+        h->stream_words = stream_words;
+        h->nsym = nsym;
+        off = align_up(off + ((uint64_t)stream_words + kStreamPad) * 4, kSectionAlign);
+        h->off_table = off;
+        off = align_up(off + (uint64_t)d->rows * (d->cols / kGroup) * 2, kSectionAlign);
+        h->off_index = off;
+        off = align_up(off + (uint64_t)d->rows * h->slots * 4, kSectionAlign);
+        h->off_codebook = off;
+        off = align_up(off + ((uint64_t)kCbSyms + (nsym + 1) / 2) * 4, kSectionAlign);
+        h->off_row_ptr = off;
+        off = align_up(off + (uint64_t)(d->rows + 1) * 4, kSectionAlign);
+        h->off_csr = off;
+        off = align_up(off + (uint64_t)d->nnz * 4 + 16, kSectionAlign);
+        h->flags = flags;
+        h->total = off;
+        return;
+    }
     off = align_up(off + (uint64_t)d->rows * h->row_words * 4, kSectionAlign);
     h->off_table = off;
     if (d->mode == DSQ_MODE_LUT_ROW)
@@ -85,12 +107,15 @@ int parse_blob(const void *packed, size_t bytes, BlobHeader *out) {
     dsq_desc d = {h.rows, h.cols, h.bits, h.mode, h.nnz};
     int rc = check_desc(&d);
     if (rc != DSQ_OK) return rc;
+    if (h.mode == DSQ_MODE_INTGRID && (h.flags != 0 || h.nsym == 0 || h.nsym > 2 * kIntGridMax + 1))
+        return DSQ_ERR_INVALID_ARG;
     BlobHeader want;
-    plan_blob(&d, &want, h.flags);
+    plan_blob(&d, &want, h.flags, h.stream_words, h.nsym);
     if (want.slots != h.slots || want.row_words != h.row_words || want.off_dense != h.off_dense ||
         want.off_table != h.off_table || want.off_row_ptr != h.off_row_ptr ||
         want.off_csr != h.off_csr || h.reserved0 != 0 || want.off_rscale != h.off_rscale ||
-        want.off_cscale != h.off_cscale || want.total != h.total || h.total > bytes)
+        want.off_cscale != h.off_cscale || want.off_index != h.off_index ||
+        want.off_codebook != h.off_codebook || want.total != h.total || h.total > bytes)
         return DSQ_ERR_INVALID_ARG;
     *out = h;
     return DSQ_OK;
@@ -137,6 +162,7 @@ static int pack_impl(const dsq_desc *d, const uint8_t *codes, const uint16_t *ta
     if (!out_bytes) return DSQ_ERR_INVALID_ARG;
     int rc = check_desc(d);
     if (rc != DSQ_OK) return rc;
+    if (d->mode == DSQ_MODE_INTGRID) return DSQ_ERR_INVALID_ARG;  // integers: dsq_pack_intgrid
     const int64_t M = d->rows, N = d->cols, nnz = d->nnz;
     const int bits = d->bits, mode = d->mode, K = 1 << bits, qmax = K - 1;
     const int64_t G = N / kGroup;

@@ -19,7 +19,13 @@
  *                          bit planes b_i = bit (i-1) of q and k+1 fp16
  *                          coefficients per group of 32 * 2^k inputs
  *                          (BPDQ page, "1. Formulation de la Grille
- *                          Variable"); the sum is exact, rounded once.
+ *                          Variable"); the sum is exact, rounded once, or
+ *   - DSQ_MODE_INTGRID:    w = fp16(scale[i][g] * q), q a signed integer with
+ *                          |q| <= 8191, an fp16 scale per group of 16 inputs:
+ *                          inliers and outliers on one unconstrained integer
+ *                          grid, the integers Huffman coded (gist.science
+ *                          2507.18553, the HPTQ bullet); packed by
+ *                          dsq_pack_intgrid, bits = 14.
  * At the positions of the outliers the dense part holds "holes" whose codes
  * still decode (to 0 when the encoder chose q = zero).
  * W_sparse holds the outliers as fp16 CSR: values / col_idx / row_ptr (SpQR
@@ -65,13 +71,14 @@ typedef enum {
     DSQ_ERR_SCRATCH_LIMIT = -7    /* dsq_gemv_noalloc: the problem needs more than its fixed scratch */
 } dsq_status;
 
-enum { DSQ_MODE_LUT_ROW = 0, DSQ_MODE_AFFINE_G16 = 1, DSQ_MODE_BITPLANE = 2 };
+enum { DSQ_MODE_LUT_ROW = 0, DSQ_MODE_AFFINE_G16 = 1, DSQ_MODE_BITPLANE = 2, DSQ_MODE_INTGRID = 3 };
 
 /* Shape and encoding of one quantized weight matrix (rows = out features M,
  * cols = in features N).  Requirements: rows >= 0; cols >= 0 and
  * cols % 16 == 0; cols <= 65535 (column indices are stored in 16 bits);
  * bits in {3, 4} for DSQ_MODE_LUT_ROW and DSQ_MODE_AFFINE_G16, in {2, 3}
- * for DSQ_MODE_BITPLANE (there also cols % (32 << bits) == 0);
+ * for DSQ_MODE_BITPLANE (there also cols % (32 << bits) == 0), 14 for
+ * DSQ_MODE_INTGRID;
  * 0 <= nnz <= rows*cols. */
 typedef struct {
     int32_t rows;
@@ -138,6 +145,25 @@ DSQ_API int dsq_pack_two_axis(const dsq_desc *d, const uint8_t *codes, const uin
                               const uint16_t *zeros, const int32_t *row_ptr, const int32_t *col_idx,
                               const uint16_t *values, const uint16_t *row_scale,
                               const uint16_t *col_scale, void *out, size_t *out_bytes);
+
+/*
+ * dsq_pack_intgrid -- pack a DSQ_MODE_INTGRID matrix: Huffman-code its
+ * integers (one canonical code per matrix, codes of at most 20 bits, an
+ * MSB-first bitstream with the bit offset of every 32-column slot so slots
+ * decode independently) and store its scales and outliers.
+ *   d       host; mode DSQ_MODE_INTGRID, bits 14.
+ *   q       host int16 [rows][cols], |q| <= 8191.
+ *   scales  host fp16 [rows][cols/16], finite.
+ *   row_ptr, col_idx, values, out, out_bytes  as for dsq_pack (an outlier
+ *           list is optional: the grid holds outliers as large integers).
+ * Returns as dsq_pack; DSQ_ERR_UNSUPPORTED when the stream would pass 2^32
+ * bits.  dsq_gemv of such a matrix runs the variable-length-decode kernel
+ * (one warp per row, lanes decoding whole slots); dsq_decode writes
+ * fp16(scale * q).
+ */
+DSQ_API int dsq_pack_intgrid(const dsq_desc *d, const int16_t *q, const uint16_t *scales,
+                             const int32_t *row_ptr, const int32_t *col_idx, const uint16_t *values,
+                             void *out, size_t *out_bytes);
 
 /*
  * dsq_blob_desc -- read the shape of a packed blob (host).  Returns

@@ -39,7 +39,9 @@ import numpy as np
 LUT = "lut"
 AFFINE = "affine"
 BITPLANE = "bitplane"
+INTGRID = "intgrid"
 GROUP = 16
+INTGRID_MAX = 8191
 
 
 def bitplane_group(bits: int) -> int:
@@ -106,6 +108,12 @@ class Problem:
             meta = self.rows * (1 << self.bits) * 2
         elif self.mode == BITPLANE:
             meta = self.rows * (self.cols // bitplane_group(self.bits)) * (self.bits + 1) * 2
+        elif self.mode == INTGRID:
+            # Huffman-coded integers: code bits, fp16 scales, slot bit offsets, codebook
+            codes = (huffman_bits(self.codes) + 7) // 8
+            nsym = int(np.unique(self.codes).size)
+            meta = self.rows * (self.cols // GROUP) * 2 + self.rows * ((self.cols + 31) // 32) * 4 \
+                + (65 + 1024) * 4 + 2 * nsym
         else:
             meta = self.rows * (self.cols // GROUP) * 4
         csr = self.nnz * 6 + (self.rows + 1) * 4
@@ -264,6 +272,36 @@ def _quantize_bitplane(Wd: np.ndarray, hole: np.ndarray, bits: int):
     return q.reshape(M, N).astype(np.uint8), f16_bits(coef)
 
 
+def huffman_bits(q: np.ndarray) -> int:
+    """Total length of an optimal Huffman code of the integers q (the
+    canonical byte count of an integer-grid matrix)."""
+    import heapq
+    _, counts = np.unique(q, return_counts=True)
+    if counts.size == 1:
+        return int(counts[0])
+    heap = [int(c) for c in counts]
+    heapq.heapify(heap)
+    total = 0
+    while len(heap) > 1:
+        a, b = heapq.heappop(heap), heapq.heappop(heap)
+        total += a + b
+        heapq.heappush(heap, a + b)
+    return total
+
+
+def _quantize_intgrid(W: np.ndarray):
+    """One unconstrained integer grid per group of 16 (the HPTQ bullet): the
+    step is half of a robust spread of the group (1.4826 * median |w|), so
+    the Gaussian bulk spans a few levels and spikes land on large integers."""
+    M, N = W.shape
+    G = W.reshape(M, N // GROUP, GROUP)
+    spread = 1.4826 * np.median(np.abs(G), axis=2)
+    s16 = f16_bits(np.where(spread > 0, spread / 2.0, 1.0))
+    sv = s16.view(np.float16).astype(np.float64)
+    q = np.clip(np.rint(G / sv[:, :, None]), -INTGRID_MAX, INTGRID_MAX).astype(np.int16)
+    return q.reshape(M, N), s16
+
+
 # ---------------------------------------------------------------- assembly
 
 def _two_axis_scales(Wd: np.ndarray, hole: np.ndarray, iters: int = 8):
@@ -305,6 +343,16 @@ def make_problem(rows: int, cols: int, bits: int, mode: str, density: float,
         W *= np.outer(np.exp(rng.normal(0.0, 0.5, M)), np.exp(rng.normal(0.0, 0.5, N)))
     nnz = round_half_up(density * M * N) if outliers != "none" else 0
     Wf = W.reshape(-1)
+    if mode == INTGRID:
+        # inliers and outliers share the grid: the spikes stay in the matrix
+        if nnz:
+            spike_pos = rng.choice(M * N, nnz, replace=False)
+            Wf[spike_pos] += rng.laplace(0.0, 0.2, nnz)
+        codes, table = _quantize_intgrid(W)
+        x = f16_bits(rng.normal(0.0, 1.0, size=(batch, N)))
+        return Problem(name=name, rows=M, cols=N, bits=14, mode=mode, codes=codes, table=table,
+                       zeros=None, row_ptr=np.zeros(M + 1, np.int32), col_idx=np.zeros(0, np.int32),
+                       values=np.zeros(0, np.uint16), x=x)
     if nnz == 0:
         pos = np.zeros(0, dtype=np.int64)
     elif outliers in ("topk", "uniform"):
@@ -394,6 +442,10 @@ CONFIGS: Dict[str, dict] = {
     "bp3": dict(rows=11008, cols=4096, bits=3, mode=BITPLANE, density=0.01,
                 outliers="uniform", seed=53, batches=(1, 2, 4),
                 about="11008x4096 3-bit-plane BPDQ (groups of 256, 4 fp16 coefficients), 1% uniform outliers"),
+    # Huffman-coded integer grid (HPTQ), inliers and spikes on one grid, same shape
+    "hq": dict(rows=11008, cols=4096, bits=14, mode=INTGRID, density=0.01,
+               outliers="uniform", seed=70, batches=(1, 2),
+               about="11008x4096 Huffman-coded integer grid (HPTQ), fp16 scale per 16, 1% Laplace spikes in the grid"),
     # SINQ two-axis scales around a non-uniform 3-bit table, same shape
     "sq3": dict(rows=11008, cols=4096, bits=3, mode=LUT, density=0.01,
                 outliers="uniform", seed=60, batches=(1, 2), two_axis=True,

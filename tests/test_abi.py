@@ -327,6 +327,96 @@ def test_two_axis_blob_sections_and_checks():
     assert lib.dsq_gemv_noalloc(ctypes.byref(desc), 256, len(blob), 16, 16, 16, None) == dsq.DSQ_ERR_INVALID_ARG
 
 
+def decode_intgrid_blob(blob: bytes):
+    """Test-only reader of an INTGRID blob, written from the format
+    description: canonical code from the codebook's per-length counts, the
+    MSB-first bitstream read code by code from each slot's bit offset."""
+    rows, cols, bits, mode = (int(v) for v in np.frombuffer(blob[16:32], np.int32))
+    S = int(np.frombuffer(blob[40:44], np.int32)[0])
+    off_dense, off_table = (int(v) for v in np.frombuffer(blob[48:64], np.uint64))
+    off_index, off_codebook = (int(v) for v in np.frombuffer(blob[120:136], np.uint64))
+    stream_words, nsym = (int(v) for v in np.frombuffer(blob[136:144], np.uint32))
+    cb = np.frombuffer(blob[off_codebook:off_codebook + 4 * (65 + 1024 + (nsym + 1) // 2)], np.uint32)
+    assert cb[0] == nsym
+    count = cb[23:44]
+    syms = np.frombuffer(cb[65 + 1024:].tobytes()[:2 * nsym], np.int16)
+    table = {}
+    code, r = 0, 0
+    for length in range(1, 21):                  # canonical: by length, then value
+        for _ in range(int(count[length])):
+            table[(length, code)] = int(syms[r])
+            code += 1
+            r += 1
+        code <<= 1
+    stream = np.frombuffer(blob[off_dense:off_dense + 4 * (stream_words + 24)], np.uint32)
+    bitstr = np.unpackbits(stream.byteswap().view(np.uint8))   # MSB-first bit order
+    idx = np.frombuffer(blob[off_index:off_index + 4 * rows * S], np.uint32).reshape(rows, S)
+    q = np.zeros((rows, cols), np.int16)
+    for i in range(rows):
+        for s in range(S):
+            pos = int(idx[i, s])
+            for c in range(min(32, cols - 32 * s)):
+                code, length = 0, 0
+                while (length, code) not in table:
+                    code = (code << 1) | int(bitstr[pos])
+                    pos += 1
+                    length += 1
+                    assert length <= 20
+                q[i, 32 * s + c] = table[(length, code)]
+    scales = np.frombuffer(blob[off_table:off_table + 2 * rows * (cols // 16)], np.uint16).reshape(rows, -1)
+    return q, scales
+
+
+@pytest.mark.parametrize("rows,cols,seed", [(9, 256, 1), (3, 48, 2), (17, 1040, 3)])
+def test_intgrid_blob_round_trip(rows, cols, seed):
+    p = synth.make_problem(rows, cols, 14, "intgrid", 0.02, "uniform", seed, 1)
+    q, scales = decode_intgrid_blob(dsq.pack_problem(p))
+    assert np.array_equal(q, p.codes) and np.array_equal(scales, p.table)
+
+
+def test_intgrid_long_codes_and_one_symbol():
+    """Skewed frequencies force codes past the 10-bit fast table (and past 20
+    bits before limiting); a matrix of one integer has a one-symbol code."""
+    rng = np.random.default_rng(8)
+    q = np.zeros((4, 4096), np.int16)
+    q.reshape(-1)[:] = np.minimum(rng.geometric(0.5, q.size) - 1, 40).astype(np.int16) * np.where(rng.random(q.size) < 0.5, -1, 1)
+    q[2, 5] = 8191
+    q[3, 7] = -8191
+    sc = np.full((4, 256), 0x3C00, np.uint16)
+    blob = dsq.pack_intgrid(4, 4096, q, sc, np.zeros(5, np.int32), np.zeros(0, np.int32), np.zeros(0, np.uint16))
+    assert np.array_equal(decode_intgrid_blob(blob)[0], q)
+    nsym = int(np.frombuffer(blob[140:144], np.uint32)[0])
+    off_cb = int(np.frombuffer(blob[128:136], np.uint64)[0])
+    max_len = int(np.frombuffer(blob[off_cb + 4:off_cb + 8], np.uint32)[0])
+    assert nsym > 20 and 10 < max_len <= 20          # codes past the fast table, limited to 20 bits
+    one = np.full((2, 64), -3, np.int16)
+    blob = dsq.pack_intgrid(2, 64, one, np.full((2, 4), 0x3C00, np.uint16), np.zeros(3, np.int32),
+                            np.zeros(0, np.int32), np.zeros(0, np.uint16))
+    assert np.array_equal(decode_intgrid_blob(blob)[0], one)
+
+
+def test_intgrid_refusals():
+    lib = dsq.library()
+    q = np.zeros((2, 32), np.int16)
+    sc = np.full((2, 2), 0x3C00, np.uint16)
+    rp = np.zeros(3, np.int32)
+    with pytest.raises(dsq.DSQError):
+        dsq.pack_intgrid(2, 32, np.full((2, 32), 8192, np.int16), sc, rp, np.zeros(0, np.int32), np.zeros(0, np.uint16))
+    with pytest.raises(dsq.DSQError):
+        dsq.pack_intgrid(2, 32, q, np.full((2, 2), 0x7C00, np.uint16), rp, np.zeros(0, np.int32), np.zeros(0, np.uint16))
+    size = ctypes.c_size_t(0)
+    d = dsq.Desc(2, 32, 13, dsq.MODE_INTGRID, 0)           # bits must be 14
+    assert lib.dsq_pack_intgrid(ctypes.byref(d), q.ctypes.data, sc.ctypes.data, rp.ctypes.data, None, None,
+                                None, ctypes.byref(size)) == dsq.DSQ_ERR_INVALID_ARG
+    d = dsq.Desc(2, 32, 14, dsq.MODE_INTGRID, 0)           # integers go through dsq_pack_intgrid only
+    assert lib.dsq_pack(ctypes.byref(d), q.ctypes.data, sc.ctypes.data, None, rp.ctypes.data, None, None,
+                        None, ctypes.byref(size)) == dsq.DSQ_ERR_INVALID_ARG
+    blob = bytearray(dsq.pack_intgrid(2, 32, q, sc, rp, np.zeros(0, np.int32), np.zeros(0, np.uint16)))
+    off_index = int(np.frombuffer(bytes(blob[120:128]), np.uint64)[0])
+    blob[off_index:off_index + 4] = np.array([1 << 30], np.uint32).tobytes()   # a slot past the stream
+    assert _create_rc(bytes(blob)) == dsq.DSQ_ERR_INVALID_ARG
+
+
 def test_three_bit_fields():
     """3-bit placement: columns 2j and 2j+1 of a word's ten sit 16 bits apart
     (one mask puts both into the two 16-bit halves); every pair lies in bits

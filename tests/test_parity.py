@@ -139,6 +139,48 @@ def test_bitplane_small_shapes(orc, bits, rows, cols):
             check_y(y, y_ref, bound, f"{rows}x{cols} bitplane k={bits} B={batch}")
 
 
+@pytest.mark.parametrize("batch", [1, 2, 5, 9])
+def test_gemv_intgrid_every_row(orc, batch):
+    """Huffman-coded integer grid (11008 x 4096, spikes in the grid): the
+    variable-length-decode kernel, every row against the oracle; the decode
+    is bit-exact."""
+    p, h = config("hq")
+    if batch == 1:
+        assert np.array_equal(to_bits(h.decode()), orc.decode(p))
+    xb = synth.f16_bits(np.random.default_rng(80 + batch).standard_normal((batch, p.cols)))
+    y = gemv(h, xb, batch)
+    y_ref, bound = oracle_all_rows(orc, p, xb)
+    check_y(y, y_ref, bound, f"hq B={batch}")
+
+
+def test_intgrid_small_cases(orc):
+    """Long codes (past the fast table), one-symbol codes, extra CSR
+    outliers, ragged row counts."""
+    import types
+    rng = np.random.default_rng(9)
+    for rows, cols in ((1, 16), (7, 48), (33, 4096), (130, 512)):
+        q = (np.minimum(rng.geometric(0.4, (rows, cols)) - 1, 60) * np.where(rng.random((rows, cols)) < 0.5, -1, 1)).astype(np.int16)
+        q.reshape(-1)[0] = 8191
+        sc = synth.f16_bits(np.exp2(rng.integers(-12, 0, (rows, cols // 16))))
+        base = synth.make_problem(rows, cols, 3, "affine", 0.02, "uniform", rows, 3)
+        p = types.SimpleNamespace(rows=rows, cols=cols, bits=14, mode="intgrid", codes=q, table=sc, zeros=None,
+                                  row_ptr=base.row_ptr, col_idx=base.col_idx, values=base.values, x=base.x)
+        with dsq.Handle(dsq.pack_problem(p)) as h:
+            assert np.array_equal(to_bits(h.decode()), orc.decode(p))
+            for batch in (1, 3):
+                y = gemv(h, p.x, batch)
+                y_ref, bound = orc.gemv(p, x=p.x[:batch])
+                check_y(y, y_ref, bound, f"intgrid {rows}x{cols} B={batch}")
+    p = types.SimpleNamespace(rows=3, cols=64, bits=14, mode="intgrid", codes=np.full((3, 64), 5, np.int16),
+                              table=np.full((3, 4), 0x3800, np.uint16), zeros=None, row_ptr=np.zeros(4, np.int32),
+                              col_idx=np.zeros(0, np.int32), values=np.zeros(0, np.uint16),
+                              x=synth.f16_bits(rng.standard_normal((1, 64))))
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        assert np.array_equal(to_bits(h.decode()), orc.decode(p))
+        y_ref, bound = orc.gemv(p)
+        check_y(gemv(h, p.x, 1), y_ref, bound, "one symbol")
+
+
 @pytest.mark.parametrize("batch", [1, 2])
 def test_gemv_two_axis_every_row(orc, batch):
     """SINQ two-axis scales around a 3-bit table matrix (11008 x 4096): the
