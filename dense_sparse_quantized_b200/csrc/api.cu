@@ -148,7 +148,7 @@ extern "C" int dsq_gemv(dsq_handle_t h, const void *x, void *y, int batch, void 
 
 extern "C" int dsq_gemv_launches(dsq_handle_t h, int batch) {
     if (!h || batch < 1) return -1;
-    if (h->view.mode == DSQ_MODE_INTGRID) return gemv_launch_count(h, batch);
+    if (h->view.mode == DSQ_MODE_INTGRID) return intgrid_launch_count(h, batch);
     int n = tc_launch_count(h, batch);
     if (n < 0 && batch > 1) n = batched_launch_count(h, batch);
     if (n < 0 && fused_launch_count(h, 1) > 0) n = batch * fused_launch_count(h, 1);

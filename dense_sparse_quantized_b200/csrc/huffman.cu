@@ -29,7 +29,7 @@ namespace dsq {
 
 namespace {
 
-constexpr size_t kIntGridXsMax = 40 * 1024;  // x staged in shared memory up to this size (with the 4 KB table, under the default 48 KB)
+constexpr size_t kIntGridXsMax = 132 * 1024;  // transposed x of the launch's activation rows (cols <= 65535: one row fits)
 
 __device__ __forceinline__ uint32_t window32(const uint32_t *__restrict__ stream, uint32_t p) {
     const uint32_t hi = __ldg(stream + (p >> 5)), lo = __ldg(stream + (p >> 5) + 1);
@@ -69,71 +69,146 @@ __device__ __forceinline__ void load_fast(uint32_t *fast, const uint32_t *cb) {
     for (int i = threadIdx.x; i < (1 << kHuffFastBits); i += blockDim.x) fast[i] = __ldg(cb + kCbFast + i);
 }
 
-// One block per output row, one thread per slot (several when the row has
-// more slots than threads): each thread decodes its slots' 32 codes, forms
-// scale * q exactly in fp32 and accumulates against x; the block adds the
-// row's CSR outliers and sums everything in a fixed order.
-// xs_stage: x of the nb rows is copied to shared memory first (when it fits
-// the launch's dynamic shared memory): a lane per slot reads x 64 bytes away
-// from its neighbour, which global loads would serve one line at a time.
+// Long codes, counted against left-justified limits: with the canonical
+// code, a window `top` starts a code longer than l bits exactly when top >=
+// lim[l] = (first code of length l + count of length l) << (32 - l), so the
+// length of a code longer than kHuffFastBits is kHuffFastBits + 1 plus the
+// number of lengths l in (kHuffFastBits, maxl) with top >= lim[l].  lim and
+// first come from the per-length counts alone (a running code), the symbol
+// index is clamped to the symbol table.
+struct LongCodes {
+    uint32_t lim[kHuffMaxLen + 1];
+    uint32_t first[kHuffMaxLen + 1];
+    uint32_t offset[kHuffMaxLen + 1];
+    uint32_t maxl, nsym;
+};
+
+__device__ void load_long_codes(LongCodes &lc, const uint32_t *cb) {
+    if (threadIdx.x == 0) {
+        const uint32_t maxl = min(__ldg(cb + 1), (uint32_t)kHuffMaxLen);
+        uint32_t code = 0;
+        for (int l = 1; l <= kHuffMaxLen; l++) {
+            const uint32_t n = l <= (int)maxl ? __ldg(cb + kCbCount + l) : 0u;
+            lc.first[l] = code;
+            lc.offset[l] = __ldg(cb + kCbOffset + l);
+            code += n;
+            lc.lim[l] = l < 32 ? code << (32 - l) : code;
+            code <<= 1;
+        }
+        lc.maxl = maxl;
+        lc.nsym = max(__ldg(cb), 1u);
+    }
+}
+
+// Per lane: a 64-bit bit buffer, most significant bit first, holding nb >= 20
+// valid bits before every code (a refill adds one stream word when nb < 32).
+struct BitReader {
+    uint64_t buf;
+    int nb;
+    const uint32_t *next;
+    __device__ __forceinline__ void start(const uint32_t *stream, uint32_t p) {
+        const uint32_t *w = stream + (p >> 5);
+        buf = ((((uint64_t)__ldg(w)) << 32) | __ldg(w + 1)) << (p & 31u);
+        nb = 64 - (int)(p & 31u);
+        next = w + 2;
+    }
+    __device__ __forceinline__ int decode(const uint32_t *fast, const LongCodes &lc, const uint16_t *syms) {
+        const uint32_t top = (uint32_t)(buf >> 32);
+        const uint32_t f = fast[top >> (32 - kHuffFastBits)];
+        uint32_t len = f >> 16;
+        int v = (int)(int16_t)(f & 0xffffu);
+        if (len == 0) {
+            len = kHuffFastBits + 1;
+            for (uint32_t l = kHuffFastBits + 1; l < lc.maxl; l++) len += top >= lc.lim[l] ? 1u : 0u;
+            const uint32_t sym = min(lc.offset[len] + (top >> (32 - len)) - lc.first[len], lc.nsym - 1);
+            v = (int)(int16_t)__ldg(syms + sym);
+        }
+        buf <<= len;
+        nb -= (int)len;
+        if (nb < 32) {
+            buf |= (uint64_t)__ldg(next++) << (32 - nb);
+            nb += 32;
+        }
+        return v;
+    }
+};
+
+// Persistent warps, one output row at a time: lane l decodes slots l, l+32,
+// ... of the row, each slot's 32 codes from its own bit offset; a group of
+// 16 codes accumulates sum q * x in fp32 and is scaled once by its fp16
+// scale; the row's CSR outliers are spread over the lanes; one fixed
+// shuffle tree sums the lanes and lane b stores y[b][row].
+// Shared memory: the fast table, the long-code limits and x of nb activation
+// rows transposed to [row b][column pair pc of the slot][slot] (one padding
+// word per line), so the lanes -- on consecutive slots -- read consecutive
+// words, staged once per block.
 template <int BC>
 __global__ void __launch_bounds__(256) intgrid_gemv_kernel(MatrixView m, const __half *__restrict__ x,
-                                                           __half *__restrict__ y, int batch, int b0,
-                                                           int xs_stage) {
-    extern __shared__ __half xs_smem[];
+                                                           __half *__restrict__ y, int batch, int b0) {
+    extern __shared__ uint32_t xs[];
     __shared__ uint32_t fast[1 << kHuffFastBits];
-    const int row = blockIdx.x;
-    const int nb = min(BC, batch - b0), N = m.cols, S = m.slots;
-    const __half *scales = reinterpret_cast<const __half *>(m.table) + (size_t)row * (N / kGroup);
+    __shared__ LongCodes lc;
+    const int N = m.cols, S = m.slots, SP = S + 1;
+    const int nb = min(BC, batch - b0);
     load_fast(fast, m.codebook);
-    const __half *xb = x + (size_t)b0 * N;
-    if (xs_stage) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(xb);
-        uint4 *dst = reinterpret_cast<uint4 *>(xs_smem);
-        for (int i = threadIdx.x; i < nb * N / 8; i += blockDim.x) dst[i] = __ldg(src + i);
-        xb = xs_smem;
+    load_long_codes(lc, m.codebook);
+    for (int i = threadIdx.x; i < BC * 16 * S; i += blockDim.x) {
+        const int b = i / (16 * S), r = i - b * 16 * S, s = r >> 4, pc = r & 15, col = 32 * s + 2 * pc;
+        uint32_t v = 0;
+        if (b < nb && col < N) v = __ldg(reinterpret_cast<const uint32_t *>(x + (size_t)(b0 + b) * N + col));
+        xs[(b * 16 + pc) * SP + s] = v;
     }
     __syncthreads();
-    float acc[BC];
+    const uint16_t *syms = reinterpret_cast<const uint16_t *>(m.codebook + kCbSyms);
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < m.rows; row += warps) {
+        const __half *scales = reinterpret_cast<const __half *>(m.table) + (size_t)row * (N / kGroup);
+        float acc[BC];
 #pragma unroll
-    for (int b = 0; b < BC; b++) acc[b] = 0.f;
-    for (int s = threadIdx.x; s < S; s += blockDim.x) {
-        uint32_t p = __ldg(m.slot_bits + (size_t)row * S + s);
-        const int ncol = min(32, N - 32 * s);  // a multiple of 16
-        for (int g = 0; g < ncol / kGroup; g++) {
-            const float sc = __half2float(scales[2 * s + g]);
-#pragma unroll 4
-            for (int c = 0; c < kGroup; c++) {
-                const int j = 32 * s + kGroup * g + c;
-                const float wv = (float)decode_one(m.dense, m.codebook, fast, p) * sc;  // exact
+        for (int b = 0; b < BC; b++) acc[b] = 0.f;
+        for (int s = lane; s < S; s += 32) {
+            BitReader br;
+            br.start(m.dense, __ldg(m.slot_bits + (size_t)row * S + s));
+            const int ngroups = min(32, N - 32 * s) / kGroup;  // 1 or 2
+            for (int g = 0; g < ngroups; g++) {
+                const float sc = __half2float(scales[2 * s + g]);
+                float ag[BC];
 #pragma unroll
-                for (int b = 0; b < BC; b++)
-                    if (b < nb) acc[b] = fmaf(wv, __half2float(xb[(size_t)b * N + j]), acc[b]);
+                for (int b = 0; b < BC; b++) ag[b] = 0.f;
+#pragma unroll
+                for (int pc = 8 * g; pc < 8 * g + 8; pc++) {
+                    const float q0 = (float)br.decode(fast, lc, syms);
+                    const float q1 = (float)br.decode(fast, lc, syms);
+#pragma unroll
+                    for (int b = 0; b < BC; b++) {
+                        const uint32_t xv = xs[(b * 16 + pc) * SP + s];
+                        const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&xv));
+                        ag[b] = fmaf(q1, xf.y, fmaf(q0, xf.x, ag[b]));
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < BC; b++) acc[b] = fmaf(sc, ag[b], acc[b]);
             }
         }
-    }
-    for (int k = m.row_ptr[row] + threadIdx.x; k < m.row_ptr[row + 1]; k += blockDim.x) {
-        const uint32_t e = __ldg(m.csr + k);
-        const float v = __half2float(__ushort_as_half((unsigned short)(e >> 16)));
-        const int j = (int)(e & 0xffffu);
+        for (int k = m.row_ptr[row] + lane; k < m.row_ptr[row + 1]; k += 32) {
+            const uint32_t e = __ldg(m.csr + k);
+            const float v = __half2float(__ushort_as_half((unsigned short)(e >> 16)));
+            const int j = (int)(e & 0xffffu), s = j >> 5, c = j & 31;
+#pragma unroll
+            for (int b = 0; b < BC; b++) {
+                const uint32_t xv = xs[(b * 16 + (c >> 1)) * SP + s];
+                acc[b] = fmaf(v, __half2float(__ushort_as_half((unsigned short)(xv >> (16 * (c & 1))))), acc[b]);
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < BC; b++) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+        }
 #pragma unroll
         for (int b = 0; b < BC; b++)
-            if (b < nb) acc[b] = fmaf(v, __half2float(x[(size_t)(b0 + b) * N + j]), acc[b]);
-    }
-    __shared__ float part[BC][8];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int b = 0; b < BC; b++) {
-        float a = acc[b];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == 0) part[b][warp] = a;
-    }
-    __syncthreads();
-    if (threadIdx.x < BC && (int)threadIdx.x < nb) {
-        float a = 0.f;
-        for (int w = 0; w < (int)(blockDim.x >> 5); w++) a += part[threadIdx.x][w];
-        y[(size_t)(b0 + threadIdx.x) * m.rows + row] = __float2half_rn(a);
+            if (lane == b && b < nb) y[(size_t)(b0 + b) * m.rows + row] = __float2half_rn(acc[b]);
     }
 }
 
@@ -235,22 +310,49 @@ int check_intgrid_contents(const void *packed, const BlobHeader &h) {
     return DSQ_OK;
 }
 
+// Activation rows per launch: x of BC rows, transposed, in shared memory
+// (BC = 4 when the batch has 3 or more rows and 4 fit, else 2, else 1).
+int intgrid_bc(int cols, int batch) {
+    const size_t per_row = (size_t)16 * (slots_of(cols) + 1) * 4;
+    const int cap = 4 * per_row <= kIntGridXsMax ? 4 : 2 * per_row <= kIntGridXsMax ? 2 : 1;
+    return std::min(cap, batch >= 3 ? 4 : batch);
+}
+
+template <int BC>
+int launch_intgrid_bc(const dsq_handle_s *h, const __half *x, __half *y, int batch, int b0, cudaStream_t st) {
+    const MatrixView &m = h->view;
+    const size_t smem = (size_t)BC * 16 * (m.slots + 1) * 4;
+    static const bool attr_ok = cudaFuncSetAttribute(intgrid_gemv_kernel<BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)kIntGridXsMax) == cudaSuccess;
+    if (!attr_ok) return DSQ_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, intgrid_gemv_kernel<BC>, 256, smem) != cudaSuccess ||
+        per_sm < 1)
+        return DSQ_ERR_CUDA;
+    const int grid = (int)std::min<int64_t>((m.rows + 7) / 8, (int64_t)per_sm * h->sm_count);
+    intgrid_gemv_kernel<BC><<<grid, 256, smem, st>>>(m, x, y, batch, b0);
+    return cudaGetLastError() == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+}
+
+int intgrid_launch_count(const dsq_handle_s *h, int batch) {
+    if (h->view.rows == 0) return 0;
+    if (h->view.cols == 0) return 1;
+    const int bc = intgrid_bc(h->view.cols, batch);
+    return (batch + bc - 1) / bc;
+}
+
 int launch_gemv_intgrid(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t st) {
     const MatrixView &m = h->view;
     if (m.rows == 0) return DSQ_OK;
     if (m.cols == 0) return launch_zero(y, (int64_t)batch * m.rows, st);
-    // one block per row, one thread per slot up to 256
-    const int threads = std::min(256, std::max(32, (m.slots + 31) / 32 * 32));
-    for (int b0 = 0; b0 < batch; b0 += 8) {
-        const int nb = std::min(8, batch - b0);
-        const size_t xbytes = (size_t)nb * m.cols * 2;
-        const int stage = xbytes <= kIntGridXsMax ? 1 : 0;
-        const size_t smem = stage ? xbytes : 0;
-        if (nb == 1) intgrid_gemv_kernel<1><<<m.rows, threads, smem, st>>>(m, x, y, batch, b0, stage);
-        else if (nb <= 4) intgrid_gemv_kernel<4><<<m.rows, threads, smem, st>>>(m, x, y, batch, b0, stage);
-        else intgrid_gemv_kernel<8><<<m.rows, threads, smem, st>>>(m, x, y, batch, b0, stage);
+    const int bc = intgrid_bc(m.cols, batch);
+    int rc = DSQ_OK;
+    for (int b0 = 0; b0 < batch && rc == DSQ_OK; b0 += bc) {
+        if (bc == 4) rc = launch_intgrid_bc<4>(h, x, y, batch, b0, st);
+        else if (bc == 2) rc = launch_intgrid_bc<2>(h, x, y, batch, b0, st);
+        else rc = launch_intgrid_bc<1>(h, x, y, batch, b0, st);
     }
-    return cudaGetLastError() == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+    return rc;
 }
 
 int launch_decode_intgrid(const dsq_handle_s *h, __half *w, cudaStream_t st) {

@@ -90,7 +90,12 @@ int gemv_launch_count(const dsq_handle_s *h, int batch);
 int launch_zero(__half *y, int64_t n, cudaStream_t stream);
 int launch_wait_timeout(const dsq_handle_s *h, cudaStream_t stream);
 // Huffman-coded integer grids (huffman.cu).
+// 4-bit row tables at 2+ activation rows on warp-level tensor cores (tc_lut.cu).
+bool tl4_covers(const dsq_handle_s *h, int batch);
+int tl4_launch_count(const dsq_handle_s *h, int batch);
+int launch_gemv_tl4(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
 int launch_gemv_intgrid(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
+int intgrid_launch_count(const dsq_handle_s *h, int batch);
 int launch_decode_intgrid(const dsq_handle_s *h, __half *w, cudaStream_t stream);
 int check_intgrid_contents(const void *packed, const BlobHeader &h);
 

@@ -155,10 +155,11 @@ def test_gemv_intgrid_every_row(orc, batch):
 
 def test_intgrid_small_cases(orc):
     """Long codes (past the fast table), one-symbol codes, extra CSR
-    outliers, ragged row counts."""
+    outliers, ragged row counts, the widest row (65520 columns: x of one
+    activation row fills the kernel's shared-memory stage)."""
     import types
     rng = np.random.default_rng(9)
-    for rows, cols in ((1, 16), (7, 48), (33, 4096), (130, 512)):
+    for rows, cols in ((1, 16), (7, 48), (33, 4096), (130, 512), (2, 65520)):
         q = (np.minimum(rng.geometric(0.4, (rows, cols)) - 1, 60) * np.where(rng.random((rows, cols)) < 0.5, -1, 1)).astype(np.int16)
         q.reshape(-1)[0] = 8191
         sc = synth.f16_bits(np.exp2(rng.integers(-12, 0, (rows, cols // 16))))
@@ -245,6 +246,37 @@ def test_batches(orc, mode, batch):
         y = gemv(h, p.x, batch)
         y_ref, bound = orc.gemv(p)
         check_y(y, y_ref, bound, f"{mode} B={batch}")
+
+
+@pytest.mark.parametrize("rows,cols", [(37, 272), (130, 1024), (16, 11008)])
+@pytest.mark.parametrize("batch", [2, 3, 7, 8, 9, 16, 17, 33])
+def test_table4_tensor_core_batches(orc, rows, cols, batch):
+    """4-bit row tables from 2 activation rows on: the centroids looked up
+    into warp-level MMA fragments (8 activation rows per launch up to 8,
+    then 16 per launch).  Ragged 16-row tiles, an odd slot count with a
+    16-column tail slot (272 columns), c3's width."""
+    p = synth.make_problem(rows, cols, 4, "lut", 0.02, "uniform", rows + cols + batch, batch)
+    with dsq.Handle(dsq.pack_problem(p)) as h:
+        y = gemv(h, p.x, batch)
+        y_ref, bound = orc.gemv(p)
+        check_y(y, y_ref, bound, f"table4 {rows}x{cols} B={batch}")
+
+
+@pytest.mark.parametrize("batch", [4, 16])
+def test_table4_tile_with_many_outlier_rounds(orc, batch):
+    """The first 16-row tile has an outlier on every column of every row
+    (16 x 16384 entries, 8464 pieces of at most 31): its piece sums are
+    folded in 17 rounds of 512; the rows after it keep a few outliers."""
+    p = synth.make_problem(40, 16384, 4, "lut", 0.001, "uniform", 12, batch)
+    rng = np.random.default_rng(3)
+    rows = [np.arange(p.cols) if i < 16 else p.col_idx[p.row_ptr[i]:p.row_ptr[i + 1]] for i in range(p.rows)]
+    rp = np.concatenate([[0], np.cumsum([len(r) for r in rows])]).astype(np.int32)
+    ci = np.concatenate(rows).astype(np.int32)
+    q = edited(p, row_ptr=rp, col_idx=ci, values=synth.f16_bits(rng.laplace(0, 0.2, ci.size)))
+    with dsq.Handle(dsq.pack_problem(q)) as h:
+        y = gemv(h, q.x, batch)
+    y_ref, bound = orc.gemv(q)
+    check_y(y, y_ref, bound, f"table4 many outlier rounds B={batch}")
 
 
 # ------------------------------------------------------------- edge cases
@@ -380,14 +412,15 @@ def test_streams_and_repeat_calls_agree():
     assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
 
 
-@pytest.mark.parametrize("mode,batch", [("affine", 1), ("affine", 16), ("lut", 1), ("lut", 4)])
-def test_back_to_back_calls_read_the_x_just_written(mode, batch):
+@pytest.mark.parametrize("mode,bits,batch", [("affine", 3, 1), ("affine", 3, 16), ("lut", 3, 1), ("lut", 3, 4),
+                                            ("lut", 4, 4), ("lut", 4, 16)])
+def test_back_to_back_calls_read_the_x_just_written(mode, bits, batch):
     """The kernels start before the previous kernel in the stream ends
     (programmatic dependent launch) and must still read the x that kernel
     wrote and write y after it: x is rewritten by a copy kernel right before
     every call, with no synchronisation, and each y must equal, bit for bit,
     the y of the same x computed in isolation."""
-    p = synth.make_problem(1024, 2048, 3, mode, 0.01, "uniform", 31, batch)
+    p = synth.make_problem(1024, 2048, bits, mode, 0.01, "uniform", 31, batch)
     rng = np.random.default_rng(5)
     xs = [to_dev(synth.f16_bits(rng.standard_normal((batch, p.cols)))) for _ in range(6)]
     with dsq.Handle(dsq.pack_problem(p)) as h:
