@@ -1030,6 +1030,8 @@ int fused_prepare(dsq_handle_s *) {
 // launch of the batched kernel (2 or 4 rows wide; 8 rows of x in registers
 // left too few warps per SM and measured slower than two passes of 4).
 int batched_launch_count(const dsq_handle_s *h, int batch) {
+    const int n_tc = tl4_launch_count(h, batch);  // 4-bit row tables: tensor cores
+    if (n_tc >= 0) return n_tc;
     B1Params p;
     size_t smem;
     const MatrixView &m = h->view;
@@ -1041,6 +1043,7 @@ int batched_launch_count(const dsq_handle_s *h, int batch) {
 }
 
 int launch_gemv_batched(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t st) {
+    if (tl4_covers(h, batch)) return launch_gemv_tl4(h, x, y, batch, st);
     if (batched_launch_count(h, batch) < 0) return DSQ_ERR_UNSUPPORTED;
     const MatrixView &m = h->view;
     for (int b0 = 0; b0 < batch; b0 += 4) {

@@ -265,8 +265,9 @@ def test_table4_tensor_core_batches(orc, rows, cols, batch):
 @pytest.mark.parametrize("batch", [4, 16])
 def test_table4_tile_with_many_outlier_rounds(orc, batch):
     """The first 16-row tile has an outlier on every column of every row
-    (16 x 16384 entries, 8464 pieces of at most 31): its piece sums are
-    folded in 17 rounds of 512; the rows after it keep a few outliers."""
+    (16 x 16384 entries: 2048 warp pieces of 128 entries), more than one
+    round of piece sums holds, so the sums are folded over several rounds;
+    the rows after it keep a few outliers."""
     p = synth.make_problem(40, 16384, 4, "lut", 0.001, "uniform", 12, batch)
     rng = np.random.default_rng(3)
     rows = [np.arange(p.cols) if i < 16 else p.col_idx[p.row_ptr[i]:p.row_ptr[i + 1]] for i in range(p.rows)]
