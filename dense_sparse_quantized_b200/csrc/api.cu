@@ -114,6 +114,8 @@ extern "C" int dsq_create(const void *packed, size_t bytes, int device, dsq_hand
     const int32_t *rp_host = (const int32_t *)((const uint8_t *)packed + hd.off_row_ptr);
     rc = build_schedule(h, rp_host);
     if (rc == DSQ_OK) rc = fused_prepare(h);
+    if (rc == DSQ_OK) rc = tl4_prepare();
+    if (rc == DSQ_OK && hd.mode == DSQ_MODE_INTGRID) rc = intgrid_prepare(h);
     if (rc == DSQ_OK) rc = tc_prepare(h, rp_host, (const uint32_t *)((const uint8_t *)packed + hd.off_csr));
     if (rc != DSQ_OK) {
         dsq_destroy(h);

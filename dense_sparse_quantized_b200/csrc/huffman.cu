@@ -319,19 +319,42 @@ int intgrid_bc(int cols, int batch) {
 }
 
 template <int BC>
+size_t intgrid_smem(const MatrixView &m) {
+    return (size_t)BC * 16 * (m.slots + 1) * 4;
+}
+
+// Blocks per launch for BC activation rows: every block resident at once
+// (one pass of persistent warps), at most one per 8 rows.
+template <int BC>
+int intgrid_grid_of(const dsq_handle_s *h, int *grid) {
+    const MatrixView &m = h->view;
+    if (cudaFuncSetAttribute(intgrid_gemv_kernel<BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kIntGridXsMax) != cudaSuccess)
+        return DSQ_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, intgrid_gemv_kernel<BC>, 256, intgrid_smem<BC>(m)) !=
+        cudaSuccess)
+        return DSQ_ERR_CUDA;
+    *grid = (int)std::min<int64_t>((m.rows + 7) / 8, (int64_t)std::max(per_sm, 0) * h->sm_count);
+    return DSQ_OK;
+}
+
+template <int BC>
 int launch_intgrid_bc(const dsq_handle_s *h, const __half *x, __half *y, int batch, int b0, cudaStream_t st) {
     const MatrixView &m = h->view;
-    const size_t smem = (size_t)BC * 16 * (m.slots + 1) * 4;
-    static const bool attr_ok = cudaFuncSetAttribute(intgrid_gemv_kernel<BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     (int)kIntGridXsMax) == cudaSuccess;
-    if (!attr_ok) return DSQ_ERR_CUDA;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, intgrid_gemv_kernel<BC>, 256, smem) != cudaSuccess ||
-        per_sm < 1)
-        return DSQ_ERR_CUDA;
-    const int grid = (int)std::min<int64_t>((m.rows + 7) / 8, (int64_t)per_sm * h->sm_count);
-    intgrid_gemv_kernel<BC><<<grid, 256, smem, st>>>(m, x, y, batch, b0);
+    const int grid = h->intgrid_grid[BC == 1 ? 0 : BC == 2 ? 1 : 2];
+    if (grid < 1) return DSQ_ERR_UNSUPPORTED;  // the shape leaves no room for a block (x of BC rows)
+    intgrid_gemv_kernel<BC><<<grid, 256, intgrid_smem<BC>(m), st>>>(m, x, y, batch, b0);
     return cudaGetLastError() == cudaSuccess ? DSQ_OK : DSQ_ERR_CUDA;
+}
+
+int intgrid_prepare(dsq_handle_s *h) {
+    if (h->view.rows == 0 || h->view.cols == 0) return DSQ_OK;
+    const int cap = intgrid_bc(h->view.cols, 4);  // activation rows whose x fits the stage
+    int rc = intgrid_grid_of<1>(h, &h->intgrid_grid[0]);
+    if (rc == DSQ_OK && cap >= 2) rc = intgrid_grid_of<2>(h, &h->intgrid_grid[1]);
+    if (rc == DSQ_OK && cap >= 4) rc = intgrid_grid_of<4>(h, &h->intgrid_grid[2]);
+    return rc;
 }
 
 int intgrid_launch_count(const dsq_handle_s *h, int batch) {

@@ -78,6 +78,7 @@ struct dsq_handle_s {
     dsq::TcPlan tc;
     int *d_status = nullptr;  // sticky error word written by kernels on a timed-out wait
     size_t device_bytes = 0;
+    int intgrid_grid[3] = {0, 0, 0};  // integer-grid blocks per launch for 1, 2, 4 activation rows
 };
 
 namespace dsq {
@@ -91,11 +92,13 @@ int launch_zero(__half *y, int64_t n, cudaStream_t stream);
 int launch_wait_timeout(const dsq_handle_s *h, cudaStream_t stream);
 // Huffman-coded integer grids (huffman.cu).
 // 4-bit row tables at 2+ activation rows on warp-level tensor cores (tc_lut.cu).
+int tl4_prepare();  // per-device kernel attributes (dsq_create, device current)
 bool tl4_covers(const dsq_handle_s *h, int batch);
 int tl4_launch_count(const dsq_handle_s *h, int batch);
 int launch_gemv_tl4(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
 int launch_gemv_intgrid(const dsq_handle_s *h, const __half *x, __half *y, int batch, cudaStream_t stream);
 int intgrid_launch_count(const dsq_handle_s *h, int batch);
+int intgrid_prepare(dsq_handle_s *h);  // per-device attributes and the launch grids (dsq_create)
 int launch_decode_intgrid(const dsq_handle_s *h, __half *w, cudaStream_t stream);
 int check_intgrid_contents(const void *packed, const BlobHeader &h);
 

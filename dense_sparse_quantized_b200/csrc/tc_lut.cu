@@ -311,9 +311,6 @@ tl4_kernel(MatrixView m, const __half *__restrict__ x, __half *__restrict__ y, i
 
 int launch_tl4(const dsq_handle_s *h, const __half *x, __half *y, int nb, cudaStream_t st) {
     const MatrixView &m = h->view;
-    static const bool attr_ok =
-        cudaFuncSetAttribute(tl4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTSmem) == cudaSuccess;
-    if (!attr_ok) return DSQ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((m.rows + 15) / 16), 1, 1);
     cfg.blockDim = dim3(kTThreads, 1, 1);
@@ -328,6 +325,12 @@ int launch_tl4(const dsq_handle_s *h, const __half *x, __half *y, int nb, cudaSt
 }
 
 }  // namespace
+
+int tl4_prepare() {
+    return cudaFuncSetAttribute(tl4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTSmem) == cudaSuccess
+               ? DSQ_OK
+               : DSQ_ERR_CUDA;
+}
 
 // 4-bit row tables, no column scales, 5 or more activation rows: 8 per launch.
 bool tl4_covers(const dsq_handle_s *h, int batch) {
