@@ -196,9 +196,13 @@ DSQ_API int dsq_create(const void *packed, size_t bytes, int device, dsq_handle_
  *          element written once, rounded to nearest from an fp32 sum.
  *   batch  >= 1.  Affine 3-bit matrices take the tensor-core path from 3
  *          rows on (from 16 when a row holds more than 256 outliers);
- *          table and bit-plane matrices take a CUDA-core kernel, 4 rows
- *          per launch;
- *          affine 4-bit matrices take the one-warp-per-row kernel.
+ *          4-bit row-table matrices take warp-level tensor-core MMAs from
+ *          5 rows on, 8 rows per launch; other table and bit-plane
+ *          matrices (and 4-bit tables at 2-4 rows) take a CUDA-core
+ *          kernel, 4 rows per launch; integer-grid matrices take the
+ *          variable-length-decode kernel, up to 4 rows per launch;
+ *          two-axis matrices at 2+ rows and affine 4-bit matrices take
+ *          the one-warp-per-row kernel.
  *   stream cudaStream_t of the handle's device, as void*.
  * x and y are the caller's and must not overlap.  The handle is read-only
  * here, so calls on several streams or threads may run concurrently.
