@@ -201,8 +201,9 @@ DSQ_API int dsq_create(const void *packed, size_t bytes, int device, dsq_handle_
  *          matrices (and 4-bit tables at 2-4 rows) take a CUDA-core
  *          kernel, 4 rows per launch; integer-grid matrices take the
  *          variable-length-decode kernel, up to 4 rows per launch;
- *          two-axis matrices at 2+ rows and affine 4-bit matrices take
- *          the one-warp-per-row kernel.
+ *          two-axis matrices (affine ones at every batch, the others
+ *          from 2 rows) and affine 4-bit matrices take the one-warp-per-
+ *          row kernel.
  *   stream cudaStream_t of the handle's device, as void*.
  * x and y are the caller's and must not overlap.  The handle is read-only
  * here, so calls on several streams or threads may run concurrently.
